@@ -1,0 +1,88 @@
+"""Seeded synthetic inputs shaped like LLM linear layers.
+
+This module only draws random numbers; it holds none of the layer's
+arithmetic, so both the CUDA path and the CPU oracle can be fed from it.
+
+Every tensor is drawn in fp32 by numpy's PCG64 generator seeded from
+``(seed, tag, shape)`` and rounded to bf16 (round-to-nearest-even). The same
+call always returns the same bytes.
+
+Workloads (linear layers ``Y = X . W^T``, X [M, K], W [N, K]):
+
+* ``tiny``: X [16, 256] ~ N(0, 1) with 1 % of entries (Bernoulli per entry)
+  multiplied by 20; W [256, 256] ~ N(0, 0.02); seed 0.
+* ``llama`` (decode and prefill shapes of Llama-3-8B): X ~ N(0, 1) with
+  ceil(0.005 K) outlier channels (columns, the same for every token) x30;
+  W ~ N(0, 0.02).
+* ``deepseek`` (DeepSeek-V3 shapes): X = z * exp(sigma_m), z ~ N(0, 1),
+  sigma_m ~ N(0, 1) per token; W = N(0, 0.01) * exp(tau_b) with
+  tau_b ~ N(0, 0.5) per 128x128 block.
+"""
+
+import math
+import zlib
+
+import numpy as np
+import torch
+
+# (N, K) of the four Llama-3-8B linears: QKV, O, gate+up, down.
+LLAMA3_8B_LINEARS = ((6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336))
+LLAMA3_8B_LM_HEAD = (128256, 4096)
+DECODE_M = (1, 8, 32, 128)
+PREFILL_M = (2048, 8192)
+# (N, K) of the DeepSeek-V3 block-scaled linears.
+DEEPSEEK_V3_LINEARS = ((2112, 7168), (24576, 7168), (7168, 7168), (4096, 7168), (7168, 2048))
+DEEPSEEK_M = (64, 4096)
+# 2:4 sparse weights and token counts.
+SPARSE_LINEARS = ((14336, 4096), (4096, 14336))
+SPARSE_M = (16, 4096)
+
+
+def _rng(seed, tag, *dims):
+    key = f"{int(seed)}|{tag}|" + ",".join(str(int(d)) for d in dims)
+    return np.random.default_rng([int(seed), zlib.crc32(key.encode())])
+
+
+def _to_bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def activations(kind, M, K, seed=0):
+    """bf16 activations [M, K] of the named workload kind."""
+    r = _rng(seed, "x-" + kind, M, K)
+    z = r.standard_normal((M, K), dtype=np.float32)
+    if kind == "tiny":
+        hit = r.random((M, K)) < 0.01
+        z = np.where(hit, z * np.float32(20.0), z)
+    elif kind == "llama":
+        n_out = math.ceil(0.005 * K)
+        ch = r.choice(K, size=n_out, replace=False)
+        z[:, ch] *= np.float32(30.0)
+    elif kind == "deepseek":
+        sigma = r.standard_normal((M, 1), dtype=np.float32)
+        z = z * np.exp(sigma)
+    else:
+        raise ValueError(f"unknown workload kind {kind!r}")
+    return _to_bf16(z)
+
+
+def weights(kind, N, K, seed=0):
+    """bf16 weights [N, K] of the named workload kind."""
+    r = _rng(seed, "w-" + kind, N, K)
+    if kind in ("tiny", "llama"):
+        w = r.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    elif kind == "deepseek":
+        w = r.standard_normal((N, K), dtype=np.float32) * np.float32(0.01)
+        nb, kb = -(-N // 128), -(-K // 128)
+        tau = r.standard_normal((nb, kb), dtype=np.float32) * np.float32(0.5)
+        spread = np.repeat(np.repeat(np.exp(tau), 128, axis=0)[:N], 128, axis=1)[:, :K]
+        w = w * spread
+    else:
+        raise ValueError(f"unknown workload kind {kind!r}")
+    return _to_bf16(w)
+
+
+def uniform_bf16(shape, lo, hi, seed=0, tag="u"):
+    """bf16 values uniform in [lo, hi) (edge-case tests)."""
+    r = _rng(seed, tag, *shape)
+    return _to_bf16(r.uniform(lo, hi, size=shape).astype(np.float32))

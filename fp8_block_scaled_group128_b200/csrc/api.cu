@@ -1,0 +1,231 @@
+// The C ABI of libfp8bs: argument validation, device checks, TMA descriptor
+// encoding and the device error word. Every entry point validates its
+// arguments before launching anything and returns an FP8BS_* status.
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fp8bs {
+
+// The device error word: 0 = fine, otherwise an FP8BS_ERR_* code recorded by a
+// kernel that gave up a bounded wait. Read and cleared by
+// fp8bs_get_device_error().
+__device__ int g_device_error = 0;
+
+namespace {
+
+std::atomic<long long> g_wait_limit{kDefaultWaitCycles};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_k(int64_t K) { return (K <= 0 || K % 128 != 0) ? FP8BS_ERR_SHAPE : FP8BS_OK; }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BS_OK : FP8BS_ERR_CUDA; }
+
+// Largest element count any single operand may have (int32 grid/TMA coordinates).
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+int current_device_info(DeviceInfo* info) {
+  static DeviceInfo cache[64];
+  static std::once_flag flags[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8BS_ERR_CUDA;
+  int st = FP8BS_OK;
+  std::call_once(flags[dev], [&] {
+    DeviceInfo d{dev, 0, 0, 0};
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      st = FP8BS_ERR_CUDA;
+    cache[dev] = d;
+  });
+  if (st != FP8BS_OK) return st;
+  *info = cache[dev];
+  if (info->sm_count <= 0) return FP8BS_ERR_CUDA;
+  if (info->major != 10 || info->minor != 0) return FP8BS_ERR_ARCH;
+  return FP8BS_OK;
+}
+
+int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                      int swizzle_128b) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return FP8BS_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle_128b ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BS_OK : FP8BS_ERR_CUDA;
+}
+
+long long wait_limit() { return g_wait_limit.load(); }
+
+int* device_error_word() {
+  static int* cache[64];
+  static std::once_flag flags[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::call_once(flags[dev], [&] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  });
+  return cache[dev];
+}
+
+}  // namespace fp8bs
+
+using namespace fp8bs;
+
+extern "C" {
+
+int fp8_quant_act_group128(const void* x_bf16, int64_t M, int64_t K, void* qa_e4m3, float* sa,
+                           void* stream) {
+  if (M < 0 || M > kMaxDim || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (M == 0) return FP8BS_OK;
+  if (!x_bf16 || !qa_e4m3 || !sa) return FP8BS_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(qa_e4m3) || !aligned16(sa)) return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_quant_act_group128(x_bf16, M, K, qa_e4m3, sa,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quant_weight_block128(const void* w_bf16, int64_t N, int64_t K, void* qw_e4m3, float* sw,
+                              void* stream) {
+  if (N < 0 || N > 65535LL * 128 || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (N == 0) return FP8BS_OK;
+  if (!w_bf16 || !qw_e4m3 || !sw) return FP8BS_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(qw_e4m3) || !aligned16(sw)) return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_quant_weight_block128(w_bf16, N, K, qw_e4m3, sw,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+int prune24_compress(const void* w_bf16, int64_t N, int64_t K, void* vals_e4m3, uint8_t* meta,
+                     float* sw, void* w_pruned_bf16, void* stream) {
+  if (N < 0 || N > 65535LL * 128 || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (N == 0) return FP8BS_OK;
+  if (!w_bf16 || !vals_e4m3 || !meta || !sw) return FP8BS_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(vals_e4m3) || !aligned16(meta) || !aligned16(sw) ||
+      (w_pruned_bf16 && !aligned16(w_pruned_bf16)))
+    return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_prune24_compress(w_bf16, N, K, vals_e4m3, meta, sw, w_pruned_bf16,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+static int check_gemm_args(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (N % 8 != 0) return FP8BS_ERR_SHAPE;  // 16-byte rows of bf16 output
+  return FP8BS_OK;
+}
+
+size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse) {
+  (void)M;
+  (void)N;
+  (void)K;
+  (void)sparse;
+  return 0;  // split-K partials are reduced in distributed shared memory
+}
+
+int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y_bf16,
+                   int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  if (int st = check_gemm_args(M, N, K)) return st;
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa || !qw || !sw || !y_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
+    return FP8BS_ERR_ALIGN;
+  if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 0)) return FP8BS_ERR_WORKSPACE;
+  (void)workspace;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_block_gemm(qa, sa, qw, sw, y_bf16, M, N, K, wait_limit(), err,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const uint8_t* meta,
+                      const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (int st = check_gemm_args(M, N, K)) return st;
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa || !vals || !meta || !sw || !y_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned16(sa) || !aligned16(vals) || !aligned16(meta) ||
+      !aligned16(sw) || !aligned16(y_bf16))
+    return FP8BS_ERR_ALIGN;
+  if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 1)) return FP8BS_ERR_WORKSPACE;
+  (void)workspace;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_sparse24_gemm(qa, sa, vals, meta, sw, y_bf16, M, N, K, wait_limit(), err,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int fp8bs_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FP8BS_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return FP8BS_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess)
+    return FP8BS_ERR_CUDA;
+  return v;
+}
+
+void fp8bs_set_wait_limit(long long cycles) {
+  g_wait_limit.store(cycles > 0 ? cycles : kDefaultWaitCycles);
+}
+
+const char* fp8bs_status_string(int status) {
+  switch (status) {
+    case FP8BS_OK: return "ok";
+    case FP8BS_ERR_NULL: return "a required pointer is NULL";
+    case FP8BS_ERR_SHAPE: return "invalid shape (K must be a positive multiple of 128; N a multiple of 8 for GEMMs)";
+    case FP8BS_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FP8BS_ERR_WORKSPACE: return "workspace too small";
+    case FP8BS_ERR_CUDA: return "CUDA call failed";
+    case FP8BS_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case FP8BS_ERR_ARCH: return "device is not sm_100 (B200)";
+    default: return "unknown status";
+  }
+}
+
+int fp8bs_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Internal launchers behind the C ABI (validated arguments only).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8bs {
+
+cudaError_t launch_quant_act_group128(const void* x, int64_t M, int64_t K, void* qa, float* sa,
+                                      cudaStream_t stream);
+cudaError_t launch_quant_weight_block128(const void* w, int64_t N, int64_t K, void* qw, float* sw,
+                                         cudaStream_t stream);
+cudaError_t launch_prune24_compress(const void* w, int64_t N, int64_t K, void* vals,
+                                    uint8_t* meta, float* sw, void* w_pruned,
+                                    cudaStream_t stream);
+
+// Dense block-scaled GEMM. Returns FP8BS_* status.
+int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,
+                      int64_t M, int64_t N, int64_t K, long long wait_limit, int* err,
+                      cudaStream_t stream);
+
+// 2:4 sparse block-scaled GEMM. Returns FP8BS_* status.
+int launch_sparse24_gemm(const void* qa, const float* sa, const void* vals, const uint8_t* meta,
+                         const float* sw, void* y, int64_t M, int64_t N, int64_t K,
+                         long long wait_limit, int* err, cudaStream_t stream);
+
+// Device address of the error word on the current device (cached per device).
+int* device_error_word();
+
+// Number of SMs and the sm major/minor of the current device (cached).
+struct DeviceInfo {
+  int device;
+  int sm_count;
+  int major;
+  int minor;
+};
+int current_device_info(DeviceInfo* info);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                      int swizzle_128b);
+
+}  // namespace fp8bs

@@ -3,9 +3,9 @@
 This module only draws random numbers; it holds none of the layer's
 arithmetic, so both the CUDA path and the CPU oracle can be fed from it.
 
-Every tensor is drawn in fp32 by numpy's PCG64 generator seeded from
+Every tensor is drawn in fp32 by torch's CPU generator seeded from
 ``(seed, tag, shape)`` and rounded to bf16 (round-to-nearest-even). The same
-call always returns the same bytes.
+call always returns the same bytes (for a given torch version).
 
 Workloads (linear layers ``Y = X . W^T``, X [M, K], W [N, K]):
 
@@ -22,7 +22,6 @@ Workloads (linear layers ``Y = X . W^T``, X [M, K], W [N, K]):
 import math
 import zlib
 
-import numpy as np
 import torch
 
 # (N, K) of the four Llama-3-8B linears: QKV, O, gate+up, down.
@@ -38,51 +37,53 @@ SPARSE_LINEARS = ((14336, 4096), (4096, 14336))
 SPARSE_M = (16, 4096)
 
 
-def _rng(seed, tag, *dims):
+def _gen(seed, tag, *dims):
     key = f"{int(seed)}|{tag}|" + ",".join(str(int(d)) for d in dims)
-    return np.random.default_rng([int(seed), zlib.crc32(key.encode())])
+    g = torch.Generator()
+    g.manual_seed((int(seed) << 32) ^ zlib.crc32(key.encode()))
+    return g
 
 
-def _to_bf16(a):
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+def _randn(g, *shape):
+    return torch.randn(*shape, generator=g, dtype=torch.float32)
 
 
 def activations(kind, M, K, seed=0):
     """bf16 activations [M, K] of the named workload kind."""
-    r = _rng(seed, "x-" + kind, M, K)
-    z = r.standard_normal((M, K), dtype=np.float32)
+    g = _gen(seed, "x-" + kind, M, K)
+    z = _randn(g, M, K)
     if kind == "tiny":
-        hit = r.random((M, K)) < 0.01
-        z = np.where(hit, z * np.float32(20.0), z)
+        hit = torch.rand(M, K, generator=g) < 0.01
+        z = torch.where(hit, z * 20.0, z)
     elif kind == "llama":
         n_out = math.ceil(0.005 * K)
-        ch = r.choice(K, size=n_out, replace=False)
-        z[:, ch] *= np.float32(30.0)
+        ch = torch.randperm(K, generator=g)[:n_out]
+        z[:, ch] *= 30.0
     elif kind == "deepseek":
-        sigma = r.standard_normal((M, 1), dtype=np.float32)
-        z = z * np.exp(sigma)
+        sigma = _randn(g, M, 1)
+        z = z * torch.exp(sigma)
     else:
         raise ValueError(f"unknown workload kind {kind!r}")
-    return _to_bf16(z)
+    return z.to(torch.bfloat16)
 
 
 def weights(kind, N, K, seed=0):
     """bf16 weights [N, K] of the named workload kind."""
-    r = _rng(seed, "w-" + kind, N, K)
+    g = _gen(seed, "w-" + kind, N, K)
     if kind in ("tiny", "llama"):
-        w = r.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+        w = _randn(g, N, K) * 0.02
     elif kind == "deepseek":
-        w = r.standard_normal((N, K), dtype=np.float32) * np.float32(0.01)
+        w = _randn(g, N, K) * 0.01
         nb, kb = -(-N // 128), -(-K // 128)
-        tau = r.standard_normal((nb, kb), dtype=np.float32) * np.float32(0.5)
-        spread = np.repeat(np.repeat(np.exp(tau), 128, axis=0)[:N], 128, axis=1)[:, :K]
+        tau = _randn(g, nb, kb) * 0.5
+        spread = torch.exp(tau).repeat_interleave(128, 0)[:N].repeat_interleave(128, 1)[:, :K]
         w = w * spread
     else:
         raise ValueError(f"unknown workload kind {kind!r}")
-    return _to_bf16(w)
+    return w.to(torch.bfloat16)
 
 
 def uniform_bf16(shape, lo, hi, seed=0, tag="u"):
     """bf16 values uniform in [lo, hi) (edge-case tests)."""
-    r = _rng(seed, tag, *shape)
-    return _to_bf16(r.uniform(lo, hi, size=shape).astype(np.float32))
+    g = _gen(seed, tag, *shape)
+    return (torch.rand(*shape, generator=g) * (hi - lo) + lo).to(torch.bfloat16)

@@ -1,0 +1,164 @@
+/*
+ * fp8bs.h - C ABI of the fine-grained (block-scaled, group-128) FP8 linear
+ * layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes Y = X . W^T for bf16 X [M, K] and W [N, K] through 8-bit
+ * floating point:
+ *
+ *   - activations are quantised per token in groups of 128 input channels,
+ *     one fp32 scale per group, computed at run time ("FP8 à granularité
+ *     fine", Hugging Face transformers docs, opening bullets and section
+ *     "Chemin rapide de DeepGEMM": activation_scheme="dynamic");
+ *   - weights are quantised per 128x128 block, one fp32 scale per block (same
+ *     page, opening bullets: weight_block_size=(128, 128); section "Format
+ *     d'échelle UE8M0": scales kept as plain float32, scale_fmt="float");
+ *   - Y[m,n] = sum_kb sA[m,kb] * sW[n/128,kb] * sum_{k in kb} qA[m,k] qW[n,k],
+ *     accumulated in fp32 and rounded to bf16;
+ *   - a 2:4 variant keeps the two largest |w| of every 4 contiguous weights
+ *     along K ("Déployer la parcimonie 2:4 avec FP8 sur Hopper", steps 2, 4,
+ *     6 and "Exemples pratiques 1"; "Combiner élagage et quantification ...",
+ *     section "La clé : la sparsité structurée 2:4") and multiplies the
+ *     compressed weights.
+ *
+ * Number format: OCP FP8 E4M3 ("fn": bias 7, no infinities, max 448).
+ * Scale of a group or block: s = amax / 448 (fp32 IEEE division). Element
+ * code: e4m3(x / s) with one fp32 IEEE division, round-to-nearest-even,
+ * saturating to +-448. A group or block whose amax is 0 has s = 0 and every
+ * element encodes as a zero carrying the element's sign (0x00 or 0x80).
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates, frees or synchronises; every call is asynchronous on
+ *     `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *   - All matrices are dense row-major, with no leading-dimension argument.
+ *   - K must be a positive multiple of 128. M == 0 or N == 0 is a no-op that
+ *     returns FP8BS_OK.
+ *   - Every data pointer must be 16-byte aligned.
+ *   - Arguments are validated before anything is launched; on an error
+ *     nothing is written and a nonzero FP8BS_ERR_* code is returned.
+ *   - A launch failure returns FP8BS_ERR_CUDA. A kernel that gave up a bounded
+ *     internal wait records FP8BS_ERR_DEVICE_TIMEOUT in a device error word,
+ *     read by fp8bs_get_device_error().
+ *   - Input and output buffers must not overlap.
+ */
+#ifndef FP8BS_H_
+#define FP8BS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8BS_OK = 0,
+  FP8BS_ERR_NULL = 1,           /* a required pointer is NULL */
+  FP8BS_ERR_SHAPE = 2,          /* K % 128 != 0, K <= 0, M/N < 0, or a size too large */
+  FP8BS_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+  FP8BS_ERR_WORKSPACE = 4,      /* workspace smaller than fp8bs_gemm_workspace_bytes() */
+  FP8BS_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
+  FP8BS_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up a bounded wait */
+  FP8BS_ERR_ARCH = 7            /* the current device is not sm_100 */
+} fp8bs_status;
+
+/*
+ * Dynamic per-token activation quantization in 1x128 groups along K
+ * ("FP8 à granularité fine", opening bullets; "Chemin rapide de DeepGEMM").
+ *
+ *   x_bf16   [M][K] bf16, input.
+ *   qa_e4m3  [M][K] E4M3 bytes, output: qa[m][k] = e4m3(x[m][k] / sa[m][k/128]).
+ *   sa       [M][K/128] fp32, output: sa[m][g] = amax_{k in group g} |x[m][k]| / 448.
+ */
+int fp8_quant_act_group128(const void* x_bf16, int64_t M, int64_t K, void* qa_e4m3, float* sa,
+                           void* stream);
+
+/*
+ * Weight quantization in 128x128 blocks ("FP8 à granularité fine", opening
+ * bullets, weight_block_size=(128, 128)).
+ *
+ *   w_bf16   [N][K] bf16, input.
+ *   qw_e4m3  [N][K] E4M3 bytes, output.
+ *   sw       [ceil(N/128)][K/128] fp32, output: block amax / 448. The last row
+ *            block covers only the valid rows when N % 128 != 0.
+ */
+int fp8_quant_weight_block128(const void* w_bf16, int64_t N, int64_t K, void* qw_e4m3, float* sw,
+                              void* stream);
+
+/*
+ * 2:4 magnitude pruning along K, then block quantization and compression
+ * ("Déployer la parcimonie 2:4 avec FP8 sur Hopper", steps 2, 4 and 6;
+ * "Combiner élagage et quantification ...", section on 2:4 sparsity).
+ *
+ * In every group of 4 contiguous weights along K the two largest |w| are kept
+ * (equal magnitudes: the lower index wins) and the other two become +0. The
+ * pruned matrix is then quantized exactly like fp8_quant_weight_block128
+ * (scales recomputed after pruning).
+ *
+ *   w_bf16         [N][K] bf16, input.
+ *   vals_e4m3      [N][K/2] E4M3 bytes, output: the two kept codes of group g
+ *                  at [n][2g] and [n][2g+1], in order of position.
+ *   meta           [N][K/8] bytes, output: byte j holds group 2j in bits 0-3
+ *                  and group 2j+1 in bits 4-7; each nibble is i0 | (i1 << 2)
+ *                  with i0 < i1 the kept positions (0..3) within the group.
+ *   sw             [ceil(N/128)][K/128] fp32, output.
+ *   w_pruned_bf16  [N][K] bf16, optional output (may be NULL): the pruned
+ *                  weights in bf16.
+ */
+int prune24_compress(const void* w_bf16, int64_t N, int64_t K, void* vals_e4m3, uint8_t* meta,
+                     float* sw, void* w_pruned_bf16, void* stream);
+
+/*
+ * Block-scaled FP8 GEMM ("FP8 à granularité fine": 1x128 activation groups
+ * against 128x128 weight blocks):
+ *   y[m][n] = bf16_rn( sum_kb sa[m][kb] * sw[n/128][kb] * sum_{k in kb} qa[m][k] * qw[n][k] )
+ * with fp32 accumulation.
+ *
+ *   qa  [M][K] E4M3, sa [M][K/128] fp32  (from fp8_quant_act_group128)
+ *   qw  [N][K] E4M3, sw [ceil(N/128)][K/128] fp32  (from fp8_quant_weight_block128)
+ *   y_bf16 [M][N] bf16, output. N must be a multiple of 8.
+ *   workspace / workspace_bytes: scratch of at least
+ *       fp8bs_gemm_workspace_bytes(M, N, K, 0) bytes (may be NULL when that is 0).
+ * Results are deterministic: the same inputs give the same bytes every call.
+ */
+int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y_bf16,
+                   int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * The block-scaled GEMM with 2:4-compressed weights (vals, meta, sw as written
+ * by prune24_compress). Same result definition as fp8_block_gemm with qw the
+ * decompressed codes (pruned positions are code 0).
+ */
+int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const uint8_t* meta,
+                      const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes needed by the GEMMs for this shape (sparse != 0: the 2:4 GEMM). */
+size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the
+ * current device (FP8BS_OK if no kernel recorded an error).
+ */
+int fp8bs_get_device_error(void* stream);
+
+/*
+ * Upper bound, in SM clock cycles, of each internal wait of the GEMM kernels
+ * (default about two seconds). cycles <= 0 restores the default. A wait that
+ * runs out makes the kernel stop early and record FP8BS_ERR_DEVICE_TIMEOUT.
+ * Intended for tests of the timeout path.
+ */
+void fp8bs_set_wait_limit(long long cycles);
+
+/* Static description of a status code. */
+const char* fp8bs_status_string(int status);
+
+/* Library version, as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int fp8bs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BS_H_ */

@@ -55,7 +55,7 @@ _SUB_STEP = 2.0 ** -9     # spacing of E4M3 subnormals (exponent field 0)
 # E4M3 codec, from the OCP 8-bit floating point definition (E4M3, "fn")
 # ----------------------------------------------------------------------------
 
-def e4m3_decode(code):
+def _e4m3_value(code):
     """Value of each E4M3 byte, as float64 (NaN for 0x7F / 0xFF).
 
     Field layout S.EEEE.MMM, exponent bias 7. Exponent field 0 is subnormal,
@@ -70,6 +70,15 @@ def e4m3_decode(code):
     mag = np.where(e == 0, m * _SUB_STEP, (1.0 + m / 8.0) * np.exp2(e - 7.0))
     mag = np.where((e == 15) & (m == 7), np.nan, mag)
     return sign * mag
+
+
+# The definition above evaluated once for each of the 256 codes.
+_DECODE_TABLE = _e4m3_value(np.arange(256, dtype=np.uint8))
+
+
+def e4m3_decode(code):
+    """Value of each E4M3 byte as float64 (``_e4m3_value``, by table lookup)."""
+    return _DECODE_TABLE[np.asarray(code, dtype=np.uint8)]
 
 
 def e4m3_encode(v):

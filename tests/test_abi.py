@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_block_scaled_group128_b200 import binding
+from fp8_block_scaled_group128_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bs.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_header_declares_the_five_operations():
+    names = _declared_functions()
+    for n in ("fp8_quant_act_group128", "fp8_quant_weight_block128", "fp8_block_gemm",
+              "prune24_compress", "fp8_sparse24_gemm"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+    assert set(_declared_functions()) <= set(binding.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.fp8bs_status_string(0) == b"ok"
+    assert b"128" in lib.fp8bs_status_string(2)
+    assert lib.fp8bs_version() >= 100
+
+
+def test_workspace_query_has_no_device_dependency(lib):
+    assert lib.fp8bs_gemm_workspace_bytes(1, 4096, 4096, 0) == 0
+
+
+BAD = ctypes.c_void_p(0x1000)
+MIS = ctypes.c_void_p(0x1004)
+
+
+@pytest.mark.parametrize("K", [0, 100, 129, -128])
+def test_shape_errors_before_any_launch(lib, K):
+    assert lib.fp8_quant_act_group128(BAD, 4, K, BAD, BAD, None) == 2
+    assert lib.fp8_quant_weight_block128(BAD, 4, K, BAD, BAD, None) == 2
+    assert lib.prune24_compress(BAD, 4, K, BAD, BAD, BAD, None, None) == 2
+    assert lib.fp8_block_gemm(BAD, BAD, BAD, BAD, BAD, 4, 8, K, None, 0, None) == 2
+    assert lib.fp8_sparse24_gemm(BAD, BAD, BAD, BAD, BAD, BAD, 4, 8, K, None, 0, None) == 2
+
+
+def test_negative_sizes_and_gemm_n_alignment(lib):
+    assert lib.fp8_quant_act_group128(BAD, -1, 128, BAD, BAD, None) == 2
+    assert lib.fp8_block_gemm(BAD, BAD, BAD, BAD, BAD, 4, 12, 128, None, 0, None) == 2
+    assert lib.fp8_block_gemm(BAD, BAD, BAD, BAD, BAD, -4, 16, 128, None, 0, None) == 2
+
+
+def test_empty_problems_are_noops(lib):
+    assert lib.fp8_quant_act_group128(None, 0, 128, None, None, None) == 0
+    assert lib.fp8_quant_weight_block128(None, 0, 128, None, None, None) == 0
+    assert lib.prune24_compress(None, 0, 128, None, None, None, None, None) == 0
+    assert lib.fp8_block_gemm(None, None, None, None, None, 0, 16, 128, None, 0, None) == 0
+    assert lib.fp8_block_gemm(None, None, None, None, None, 5, 0, 128, None, 0, None) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    assert lib.fp8_quant_act_group128(None, 4, 128, BAD, BAD, None) == 1
+    assert lib.fp8_quant_act_group128(MIS, 4, 128, BAD, BAD, None) == 3
+    assert lib.fp8_block_gemm(BAD, BAD, BAD, None, BAD, 4, 8, 128, None, 0, None) == 1
+    assert lib.fp8_block_gemm(BAD, BAD, MIS, BAD, BAD, 4, 8, 128, None, 0, None) == 3
+    assert lib.prune24_compress(BAD, 4, 128, BAD, BAD, BAD, MIS, None) == 3

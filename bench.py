@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Benchmark of the fine-grained FP8 linear-layer path on B200.
+
+One step = one pass of the whole path over the decode-shaped Llama-3-8B
+linears ((N, K) = QKV (6144, 4096), O (4096, 4096), gate+up (28672, 4096),
+down (4096, 14336); tokens M in {1, 8, 32, 128}):
+
+  1. weight quantization of the four bf16 weights (128x128 blocks)
+  2. 2:4 prune + compress of the four weights
+  3. for each M, for each linear: activation quantization (1x128 groups),
+     dense block-scaled GEMM, 2:4 sparse block-scaled GEMM
+
+The metric is HBM throughput of the step (algorithmic bytes of every launch /
+device time), with the dominant kernel's roofline fraction against the
+measured copy bandwidth. Inputs are seeded synthetic bf16 tensors; the
+per-step working set (~2.7 GB) is far larger than L2 and every weight is
+re-read only after more than L2's worth of other traffic. Every launch is
+captured once in its own CUDA graph and replayed, with one CUDA event between
+consecutive launches, so host launch cost stays out of the device timing.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (replicas, weak scaling; no collective on the data path):
+  python -m torch.distributed.run --nnodes=1 --nproc-per-node N \
+      --master-addr 127.0.0.1 --master-port P bench.py --gpus N
+"""
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "block-scaled FP8 GEMM TFLOP/s and decode GB/s, % of B200 roofline"
+UNIT = "GB/s"
+WORKLOAD = "decode-shaped Llama-3-8B linears, M in {1,8,32,128}"
+LINEARS = ((6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336))
+TOKENS = (1, 8, 32, 128)
+FALLBACK_HBM_GBS = 6650.0
+KERNELS = ("quant_weight", "prune24", "quant_act", "dense_gemm", "sparse_gemm")
+# Rows of the path the step runs (the 2:4 sparse GEMM joins once it exists).
+ROWS = ("quant_weight", "prune24", "quant_act", "dense_gemm")
+
+
+# ----------------------------------------------------------------- bytes --
+
+def kernel_bytes(kind, M, N, K):
+    """Algorithmic bytes of one launch: every input read once, every output
+    written once (E4M3 = 1 B, bf16 = 2 B, scale = 4 B, metadata = K/8 B/row)."""
+    KB, NB = K // 128, -(-N // 128)
+    if kind == "quant_act":
+        return 2 * M * K + M * K + 4 * M * KB
+    if kind == "quant_weight":
+        return 2 * N * K + N * K + 4 * NB * KB
+    if kind == "prune24":
+        return 2 * N * K + N * K // 2 + N * K // 8 + 4 * NB * KB
+    if kind == "dense_gemm":
+        return N * K + 4 * NB * KB + M * K + 4 * M * KB + 2 * M * N
+    if kind == "sparse_gemm":
+        return N * K // 2 + N * K // 8 + 4 * NB * KB + M * K + 4 * M * KB + 2 * M * N
+    raise ValueError(kind)
+
+
+def step_launches():
+    """(kind, M, N, K) of every launch of one step, in issue order."""
+    out = [("quant_weight", 0, N, K) for N, K in LINEARS]
+    out += [("prune24", 0, N, K) for N, K in LINEARS]
+    for M in TOKENS:
+        for N, K in LINEARS:
+            out += [("quant_act", M, 0, K), ("dense_gemm", M, N, K), ("sparse_gemm", M, N, K)]
+    return [l for l in out if l[0] in ROWS]
+
+
+def step_bytes():
+    return sum(kernel_bytes(*l) for l in step_launches())
+
+
+# ------------------------------------------------------------ GPU step --
+
+class Step:
+    """Device buffers of one step and the launches through the C ABI."""
+
+    def __init__(self, device, seed=0):
+        from fp8_block_scaled_group128_b200 import synth
+        self.dev = device
+        self.w = {}
+        self.x = {}
+        for N, K in LINEARS:
+            self.w[(N, K)] = synth.weights("llama", N, K, seed=seed).to(device)
+        for M in TOKENS:
+            for K in sorted({K for _, K in LINEARS}):
+                self.x[(M, K)] = synth.activations("llama", M, K, seed=seed).to(device)
+        e = lambda *s, dt: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
+        self.qw, self.sw, self.vals, self.meta, self.sws = {}, {}, {}, {}, {}
+        for N, K in LINEARS:
+            NB, KB = -(-N // 128), K // 128
+            self.qw[(N, K)] = e(N, K, dt=torch.uint8)
+            self.sw[(N, K)] = e(NB, KB, dt=torch.float32)
+            self.vals[(N, K)] = e(N, K // 2, dt=torch.uint8)
+            self.meta[(N, K)] = e(N, K // 8, dt=torch.uint8)
+            self.sws[(N, K)] = e(NB, KB, dt=torch.float32)
+        self.qa, self.sa, self.y, self.ys = {}, {}, {}, {}
+        for M in TOKENS:
+            for N, K in LINEARS:
+                self.qa[(M, K)] = e(M, K, dt=torch.uint8)
+                self.sa[(M, K)] = e(M, K // 128, dt=torch.float32)
+                self.y[(M, N, K)] = e(M, N, dt=torch.bfloat16)
+                self.ys[(M, N, K)] = e(M, N, dt=torch.bfloat16)
+
+    def launches(self):
+        """(kind, thunk) for every launch of one step, in issue order."""
+        from fp8_block_scaled_group128_b200 import binding as fb
+        out = []
+        for N, K in LINEARS:
+            out.append(("quant_weight", lambda N=N, K=K: fb.fp8_quant_weight_block128(
+                self.w[(N, K)], qw=self.qw[(N, K)], sw=self.sw[(N, K)])))
+        for N, K in LINEARS:
+            out.append(("prune24", lambda N=N, K=K: fb.prune24_compress(
+                self.w[(N, K)], vals=self.vals[(N, K)], meta=self.meta[(N, K)],
+                sw=self.sws[(N, K)])))
+        for M in TOKENS:
+            for N, K in LINEARS:
+                out.append(("quant_act", lambda M=M, K=K: fb.fp8_quant_act_group128(
+                    self.x[(M, K)], qa=self.qa[(M, K)], sa=self.sa[(M, K)])))
+                out.append(("dense_gemm", lambda M=M, N=N, K=K: fb.fp8_block_gemm(
+                    self.qa[(M, K)], self.sa[(M, K)], self.qw[(N, K)], self.sw[(N, K)],
+                    y=self.y[(M, N, K)])))
+                out.append(("sparse_gemm", lambda M=M, N=N, K=K: fb.fp8_sparse24_gemm(
+                    self.qa[(M, K)], self.sa[(M, K)], self.vals[(N, K)], self.meta[(N, K)],
+                    self.sws[(N, K)], y=self.ys[(M, N, K)])))
+        return [(k, f) for k, f in out if k in ROWS]
+
+    def run(self):
+        """Issue one step eagerly on the current stream."""
+        for _, f in self.launches():
+            f()
+
+    def host_inputs(self):
+        """Pinned host copies of the step's inputs (for the end-to-end run)."""
+        return ({k: v.cpu().pin_memory() for k, v in self.w.items()},
+                {k: v.cpu().pin_memory() for k, v in self.x.items()})
+
+
+# --------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons
+    while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = open(os.devnull if False else "/tmp/fp8bs_clocks_%d.csv" % os.getpid(), "w+")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.out is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.out.flush()
+        self.out.seek(0)
+        rows = [l.strip().split(", ") for l in self.out.read().splitlines() if l.strip()]
+        name = self.out.name
+        self.out.close()
+        try:
+            os.remove(name)
+        except OSError:
+            pass
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- helpers --
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash():
+    """Hash of the CUDA sources, to tell whether recorded ncu traffic is stale."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_block_scaled_group128_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind):
+    """Per-launch DRAM bytes of `kind` on this workload from the committed ncu
+    summary, or None if absent or taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != source_hash():
+        return None
+    v = d.get("kernels", {}).get(kind)
+    return None if v is None else float(v["dram_bytes_per_launch"])
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value, world):
+    """Max of a float over all ranks (identity for one process)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU side --
+
+def oracle_sample(budget_s=15.0):
+    """Time the CPU oracle on a bounded sample of the step: the O-projection
+    linear (4096 x 4096) through all five stages at M = 8. Returns
+    (GB/s, seconds, description, threads)."""
+    import numpy as np
+    import oracle
+    from fp8_block_scaled_group128_b200 import synth
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        limiter = None
+    N, K, M = 4096, 4096, 8
+    w = synth.weights("llama", N, K, seed=0)
+    x = synth.activations("llama", M, K, seed=0)
+    byts = sum(kernel_bytes(k, 0 if k in ("quant_weight", "prune24") else M,
+                            0 if k == "quant_act" else N, K) for k in ROWS)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        qw, sw = oracle.quant_weight_block128(w)
+        vals, meta, sws, _ = oracle.prune24_compress(w)
+        qa, sa = oracle.quant_act_group128(x)
+        y = oracle.block_gemm(qa, sa, qw, sw)
+        ys = oracle.sparse24_gemm(qa, sa, vals, meta, sws) if "sparse_gemm" in ROWS else None
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    del y, ys, np
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    desc = (f"O-proj linear N=K=4096 at M=8 through the step's stages "
+            f"({', '.join(ROWS)}), {reps} repetition(s), 1 thread")
+    return byts * reps / el / 1e9, el, desc, 1
+
+
+# ---------------------------------------------------------------- arms --
+
+def run_ours(args, rank, world, local):
+    from fp8_block_scaled_group128_b200 import binding as fb
+    from fp8_block_scaled_group128_b200.build import build
+    if rank == 0 or not os.path.exists(fb.LIB_PATH):
+        build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fb.lib()
+    step = Step(dev, seed=rank)
+    stream = torch.cuda.Stream(dev)
+    launches = step_launches()
+    per_step_launches = len(launches)
+
+    # eager warm-up (also runs the one-time per-device setup of the library)
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            step.run()
+    stream.synchronize()
+    assert fb.get_device_error(stream) == 0
+
+    # One CUDA graph per launch (the host only replays graphs); one event is
+    # recorded on the stream between consecutive launches, so every launch's
+    # device time is measured live over the timed region.
+    graphs = []
+    for kind, fn in step.launches():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        graphs.append((kind, g))
+    stream.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for _, g in graphs:
+                g.replay()
+    torch.cuda.synchronize()
+
+    L = len(graphs)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * L + 1)]
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            evs[0].record()
+            j = 1
+            for _ in range(args.steps):
+                for _, g in graphs:
+                    g.replay()
+                    evs[j].record()
+                    j += 1
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = evs[0].elapsed_time(evs[-1])
+    kernel_ms = {k: 0.0 for k in ROWS}
+    for j in range(1, len(evs)):
+        kernel_ms[graphs[(j - 1) % L][0]] += evs[j - 1].elapsed_time(evs[j]) / args.steps
+    assert fb.get_device_error(stream) == 0
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+
+    sb = step_bytes()
+    value = sb * world / (ms_step * 1e-3) / 1e9
+    hbm_peak, peak_kind = measured_peaks()
+
+    breakdown = {}
+    for k in ROWS:
+        kb = sum(kernel_bytes(*l) for l in launches if l[0] == k)
+        n = sum(1 for l in launches if l[0] == k)
+        ms = kernel_ms[k]
+        breakdown[k] = {"launches": n, "ms": round(ms, 4),
+                        "GB/s": round(kb / (ms * 1e-3) / 1e9, 1) if ms > 0 else None}
+    dominant = max(ROWS, key=lambda k: kernel_ms[k])
+    dom_launches = [l for l in launches if l[0] == dominant]
+    dom_bytes_per_launch = sum(kernel_bytes(*l) for l in dom_launches) / len(dom_launches)
+    dom_ms_per_launch = kernel_ms[dominant] / len(dom_launches)
+    achieved = dom_bytes_per_launch / (dom_ms_per_launch * 1e-3) / 1e9
+    traffic = recorded_traffic(dominant)
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
+                "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "traffic": traffic}
+
+    # end to end: pinned host inputs -> device, the step through the C ABI,
+    # device -> host read of every output Y
+    h_w, h_x = step.host_inputs()
+    h2d = sum(t.numel() * t.element_size() for t in h_w.values()) + \
+        sum(t.numel() * t.element_size() for t in h_x.values())
+    d2h = sum(t.numel() * t.element_size() for t in step.y.values()) + \
+        sum(t.numel() * t.element_size() for t in step.ys.values())
+    out_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in step.y.items()}
+    outs_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in step.ys.items()}
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_once():
+        for k, v in h_w.items():
+            step.w[k].copy_(v, non_blocking=True)
+        for k, v in h_x.items():
+            step.x[k].copy_(v, non_blocking=True)
+        step.run()
+        for k, v in step.y.items():
+            out_host[k].copy_(v, non_blocking=True)
+        for k, v in step.ys.items():
+            outs_host[k].copy_(v, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_once()
+    stream.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(e2e_steps):
+            e2e_once()
+        e1.record()
+    stream.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e = {"value": round(sb * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+           "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded bf16, Llama-3-8B linear shapes; see DESIGN.md)",
+        "config": {"workload": WORKLOAD, "rows": list(ROWS), "linears_NK": [list(l) for l in LINEARS],
+                   "tokens_M": list(TOKENS), "global_batch": sum(TOKENS) * world,
+                   "step_bytes": sb, "launches_per_step": per_step_launches,
+                   "parallelism": f"replicas x{world} (token data parallel, no collective)",
+                   "l2": "working set per step ~2.7 GB >> 126 MB L2; every weight is re-read "
+                         "only after >126 MB of other traffic; CUDA-graph replay"},
+        "roofline": roofline,
+        "kernels": breakdown,
+        "e2e": e2e,
+        "gpu_launches": per_step_launches * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el, desc, cores = oracle_sample(args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores,
+                                  "kind": "oracle", "sample": desc, "seconds": round(el, 2)}
+    del graphs
+    return result
+
+
+def run_reference(args, rank, world):
+    """The oracle (numpy, fp64 GEMM) on the host cores, bounded samples."""
+    if rank != 0:
+        return None
+    samples = []
+    for _ in range(max(0, args.warmup)):
+        oracle_sample(budget_s=0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, el, desc, cores = oracle_sample(budget_s=min(args.cpu_budget, 10.0))
+        samples.append(v)
+    el_all = time.perf_counter() - t0
+    v = statistics.mean(samples)
+    sb = step_bytes()
+    ms = sb / (v * 1e9) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 oracle (fp32 quantization arithmetic)",
+        "data": "synthetic (seeded bf16)",
+        "config": {"workload": WORKLOAD, "sample": desc, "wall_s": round(el_all, 1)},
+        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the CPU baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_info()
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_ours(args, rank, world, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

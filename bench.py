@@ -48,8 +48,8 @@ LINEARS = ((6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336))
 TOKENS = (1, 8, 32, 128)
 FALLBACK_HBM_GBS = 6650.0
 KERNELS = ("quant_weight", "prune24", "quant_act", "dense_gemm", "sparse_gemm")
-# Rows of the path the step runs (the 2:4 sparse GEMM joins once it exists).
-ROWS = ("quant_weight", "prune24", "quant_act", "dense_gemm")
+# Rows of the path the step runs.
+ROWS = KERNELS
 
 
 # ----------------------------------------------------------------- bytes --

@@ -73,7 +73,7 @@ int current_device_info(DeviceInfo* info) {
 
 int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                      int swizzle_128b) {
+                      TmapSwizzle swizzle) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return FP8BS_ERR_CUDA;
   const cuuint64_t dims[2] = {inner, outer};
@@ -83,7 +83,9 @@ int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t 
   const CUresult r = fn(static_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                         const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle_128b ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle == kSwizzle128B  ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FP8BS_OK : FP8BS_ERR_CUDA;
 }

@@ -152,6 +152,25 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
+// 2:4 sparse A: D[tmem] (+)= A[smem desc, compressed] * B[smem desc]^T with
+// the A metadata read from TMEM at `e_tmem` (kind::f8f6f4, one CTA).
+__device__ __forceinline__ void mma_sp_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t e_tmem, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Copy 128 rows x 16 bytes from shared memory (matrix descriptor) into TMEM:
+// row r lands in lane r, 4 consecutive 32-bit columns from `taddr`.
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // The mbarrier at `bar` gets one arrival once every tcgen05 operation issued
 // so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -192,9 +211,24 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same for rows of 64 bytes with 64-byte swizzling (8-row atoms of 512
+// bytes, swizzle mode 4).
+__device__ __forceinline__ uint64_t sw64_kmajor_desc(uint32_t smem_addr) {
+  return static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(512 >> 4) << 32) | (1ull << 46) | (4ull << 61);
+}
+
+// Un-swizzled K-major descriptor: 8-row core matrices of 16-byte rows stored
+// contiguously (128 B), consecutive core matrices along M `sbo_bytes` apart.
+__device__ __forceinline__ uint64_t noswizzle_kmajor_desc(uint32_t smem_addr, uint32_t sbo_bytes) {
+  return static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4) | (1ull << 16) |
+         (static_cast<uint64_t>(sbo_bytes >> 4) << 32) | (1ull << 46);
+}
+
 // Instruction descriptor, kind::f8f6f4: E4M3 x E4M3 -> F32, both operands
-// K-major, no negation, dense. D format bits 4-5 (1 = F32), A/B formats bits
-// 7-9 / 10-12 (0 = E4M3), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+// K-major, no negation. D format bits 4-5 (1 = F32), A/B formats bits 7-9 /
+// 10-12 (0 = E4M3), N >> 3 in bits 17-22, M >> 4 in bits 24-28; bit 2 marks
+// a 2:4 sparse A (set by the caller), bits 0-1 select the metadata part (0).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }

@@ -1,0 +1,541 @@
+// The block-scaled FP8 GEMM kernel on tcgen05 tensor cores (shared by the
+// dense and the 2:4 sparse entry points).
+//
+//   Y[m,n] = bf16_rn( sum_kb sA[m,kb] * sW[n/128,kb] * sum_{k in kb} qA[m,k] qW[n,k] )
+//
+// ("FP8 à granularité fine": 1x128 activation groups against 128x128 weight
+// blocks, fp32 scales.) The scales change every 128-deep K-block, so the
+// tensor cores cannot accumulate across K-blocks by themselves. Each K-block
+// is one "partial" MMA chain written fresh into TMEM, and the epilogue warps
+// promote it into fp32 register accumulators multiplied by sA * sW:
+//
+//   warp 0 (one lane)  TMA producer: K-block tiles -> shared memory, a
+//                      kStages-deep ring of mbarriers.
+//   warp 1 (one lane)  MMA issuer: per K-block, 4 x tcgen05.mma kind::f8f6f4
+//                      (K = 32 each), or for 2:4 weights one tcgen05.cp of the
+//                      metadata into TMEM and 2 x tcgen05.mma.sp (logical K =
+//                      64 each), into TMEM partial buffer (kb % 2); commits
+//                      free the smem stage and signal the partial.
+//   warps 4..          promotion / epilogue: tcgen05.ld the partial, FMA into
+//                      registers with the K-block's scale product, hand the
+//                      TMEM buffer back; at the end of a tile, round to bf16
+//                      and store (or reduce split-K partials over the cluster).
+//
+// Operand orders:
+//   kSwap = false (prefill, dense): MMA rows = tokens (128), MMA cols =
+//     weight rows (BN = 256).
+//   kSwap = true (decode, and every 2:4 launch): MMA rows = 128 weight rows,
+//     MMA cols = tokens (BN = 16..256). When the weight tiles alone do not
+//     fill the GPU, K is split over a thread-block cluster of `splits` CTAs
+//     that sum their partial tiles through distributed shared memory in rank
+//     order, so results are deterministic and no global scratch is used.
+// Without a K split the CTAs are persistent: CTA y walks tiles y, y+gridDim.y...
+//
+// Every mbarrier wait is bounded; a wait that runs out records
+// FP8BS_ERR_DEVICE_TIMEOUT, and the CTA drains its own copies and MMAs in
+// flight, frees TMEM and returns.
+#pragma once
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fp8bs {
+
+namespace gemm_detail {
+
+constexpr int kBK = 128;               // K-block depth = one scale group, 128 bytes of E4M3
+constexpr int kGroupRows = 16;         // tile raster: row tiles per group (L2 reuse)
+constexpr int kEBytes = 128 * 16;      // sparse: metadata of one 128x128 block, 16 B per row
+
+struct GemmArgs {
+  const float* sa;      // [M][KB]
+  const float* sw;      // [NB][KB]
+  __nv_bfloat16* y;     // [M][N]
+  int M, N, KB, NB;
+  int row_tiles;        // tiles along the MMA M side (128 rows each)
+  int col_tiles;        // tiles along the MMA N side (BN rows each)
+  int splits;           // K splits = cluster size along x
+  long long wait_limit; // bound of each mbarrier wait, SM cycles
+  int* err;             // device error word
+};
+
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
+struct Cfg {
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
+  static_assert((BN & (BN - 1)) == 0, "BN is a power of two (TMEM allocation)");
+  static_assert(!kSparse || kSwap, "the 2:4 operand is the weight, on the MMA M side");
+  // A stage: 128 rows x 128 B (dense, 128 B swizzle) or 128 rows x 64 B of
+  // compressed 2:4 values (64 B swizzle); B stage: BN rows x 128 B.
+  static constexpr int kABytes = kSparse ? 128 * kBK / 2 : 128 * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes + (kSparse ? kEBytes : 0);
+  static constexpr int kThreads = 128 * (1 + kEpiWG);
+  static constexpr int kCols = BN / kEpiWG;  // accumulator columns per epilogue thread
+  static_assert(kCols % 16 == 0 && kCols <= 128, "epilogue column split");
+  // TMEM: two partial buffers of BN columns, then (sparse) two metadata
+  // buffers of 4 columns; the allocation is a power of two >= 32.
+  static constexpr int kTmemUsed = 2 * BN + (kSparse ? 8 : 0);
+  static constexpr int kTmemCols =
+      kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
+  static_assert(kTmemUsed <= 512, "TMEM has 512 columns");
+  static constexpr uint32_t kIdesc = idesc_e4m3_f32(128, BN) | (kSparse ? (1u << 2) : 0u);
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kStages * kABytes;
+  static constexpr int kOffE = kOffB + kStages * kBBytes;
+  static constexpr int kOffBar = kOffE + (kSparse ? kStages * kEBytes : 0);
+  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmem + 4;
+  static constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + slack to align the base
+  // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
+  static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage buffers stay 1024-aligned");
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int row_tiles, int col_tiles, int& rt,
+                                            int& ct) {
+  const int per_group = kGroupRows * col_tiles;
+  const int g = tile / per_group;
+  const int first = g * kGroupRows;
+  const int rows = min(kGroupRows, row_tiles - first);
+  const int local = tile - g * per_group;
+  rt = first + local % rows;
+  ct = local / rows;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
+__global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThreads, 1)
+    block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                      const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_e, const GemmArgs args) {
+  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG>;
+  constexpr int kABytes = C::kABytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sm_a = smem + C::kOffA;
+  uint8_t* sm_b = smem + C::kOffB;
+  uint8_t* sm_e = smem + C::kOffE;  // sparse only: metadata stages
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int kb0 = static_cast<int>(static_cast<long long>(split) * args.KB / args.splits);
+  const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * args.KB / args.splits);
+  const int num_tiles = args.row_tiles * args.col_tiles;
+  const long long limit = args.wait_limit;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4 * kEpiWG);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+    if constexpr (kSparse) tma_prefetch_desc(&tmap_e);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Registers of the epilogue threads that outlive the role loop (split-K).
+  float acc[C::kCols];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer --
+      uint64_t pol_a = 0, pol_b = 0;
+      if constexpr (kSwap) {
+        pol_a = policy_evict_first();
+        pol_b = policy_evict_last();
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int tile = blockIdx.y; tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+        int rt, ct;
+        tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
+            record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          if constexpr (kSparse) {
+            // compressed values: 64 B per row per K-block; metadata: 16 B per row
+            tma_load_2d_hint(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * (kBK / 2),
+                             rt * 128, pol_a);
+            tma_load_2d_hint(sm_e + stage * kEBytes, &tmap_e, &full[stage], kb * 16, rt * 128,
+                             pol_a);
+            tma_load_2d_hint(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK,
+                             ct * BN, pol_b);
+          } else if constexpr (kSwap) {
+            // decode: weights are streamed once, activations are shared by all CTAs
+            tma_load_2d_hint(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * kBK, rt * 128,
+                             pol_a);
+            tma_load_2d_hint(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK,
+                             ct * BN, pol_b);
+          } else {
+            tma_load_2d(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * kBK, rt * 128);
+            tma_load_2d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK, ct * BN);
+          }
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Every copy issued must have landed before shared memory is reused or
+      // the CTA exits (matters only when a consumer stopped early).
+      const int pending = issued < kStages ? issued : kStages;
+      for (int i = 0; i < pending; ++i) {
+        int s = stage - 1 - i;
+        uint32_t ph = phase;
+        if (s < 0) {
+          s += kStages;
+          ph ^= 1u;
+        }
+        mbar_wait(&full[s], ph, kDefaultWaitCycles);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // -------------------------------------------------------- MMA issuer --
+      int stage = 0;
+      uint32_t phase = 0;
+      int tb = 0;
+      uint32_t tphase = 0;
+      uint32_t e_buf = 0;  // sparse: TMEM metadata buffer, alternating per K-block
+      bool ok = true;
+      for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!mbar_wait(&full[stage], phase, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
+          const uint32_t a0 = smem_u32(sm_a + stage * kABytes);
+          const uint32_t b0 = smem_u32(sm_b + stage * C::kBBytes);
+          if constexpr (kSparse) {
+            // metadata of this K-block -> TMEM (4 columns, lane = weight row),
+            // then two sparse MMAs of logical depth 64 (32 compressed bytes
+            // of A and 64 bytes of B each), reading 2 metadata columns each
+            const uint32_t te = tmem_base + static_cast<uint32_t>(2 * BN) + 4u * e_buf;
+            e_buf ^= 1u;
+            tmem_cp_128x128b(te, noswizzle_kmajor_desc(smem_u32(sm_e + stage * kEBytes), 128));
+#pragma unroll
+            for (int k = 0; k < kBK / 64; ++k) {
+              mma_sp_f8f6f4(d, sw64_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 64 * k),
+                            te + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < kBK / 32; ++k) {
+              mma_f8f6f4(d, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                         C::kIdesc, k > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[tb]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          tb ^= 1;
+          if (tb == 0) tphase ^= 1u;
+        }
+      }
+      if (!ok) {
+        record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+        *abort_flag = 1;
+      }
+      // All MMAs issued must be complete before TMEM is freed.
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, kDefaultWaitCycles);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------- promotion / epilogue --
+    const int wg = (warp - 4) >> 2;     // epilogue warpgroup
+    const int quarter = warp & 3;       // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int row = quarter * 32 + lane;
+    const int col0 = wg * C::kCols;
+    const int KB = args.KB;
+    int tb = 0;
+    uint32_t tphase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+      int rt, ct;
+      tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
+#pragma unroll
+      for (int i = 0; i < C::kCols; ++i) acc[i] = 0.0f;
+
+      // Scale sources. Prefill: one scale per thread and K-block,
+      // sA[m,kb] * sW[nb,kb]. Decode (swap): one scale per column (token),
+      // sW[rt,kb] * sA[tok,kb]; lane l fetches the scale of column (32c + l)
+      // of each 32-column chunk c and the warp shares them by shuffles.
+      const int m = rt * 128 + row;
+      const int nb = (ct * BN + col0) / 128;
+      const float* sa_row = args.sa + static_cast<int64_t>(m < args.M ? m : 0) * KB;
+      const bool row_ok = !kSwap && m < args.M && nb < args.NB;
+      constexpr int kChunks = C::kCols / 32 > 0 ? C::kCols / 32 : 1;
+      int tok_l[kChunks];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) tok_l[c] = ct * BN + col0 + 32 * c + lane;
+
+      auto load_scales = [&](int kb, float* sc) {
+        if constexpr (!kSwap) {
+          sc[0] = row_ok ? sa_row[kb] * args.sw[static_cast<int64_t>(nb) * KB + kb] : 0.0f;
+        } else {
+          const float swv = args.sw[static_cast<int64_t>(rt) * KB + kb];
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            const bool tok_ok = tok_l[c] < args.M && (32 * c + lane) < C::kCols;
+            sc[c] = tok_ok ? swv * args.sa[static_cast<int64_t>(tok_l[c]) * KB + kb] : 0.0f;
+          }
+        }
+      };
+      float sc_cur[kChunks], sc_next[kChunks];
+      if (kb0 < kb1) load_scales(kb0, sc_cur);
+
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (kb + 1 < kb1) load_scales(kb + 1, sc_next);
+        if (!mbar_wait(&tfull[tb], tphase, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
+#pragma unroll
+        for (int c = 0; c < C::kCols; c += 32) {
+          float v0[16], v1[16];
+          tmem_ld16(taddr + c, v0);
+          if (c + 16 < C::kCols) tmem_ld16(taddr + c + 16, v1);
+          tmem_wait_ld();
+          if constexpr (!kSwap) {
+            const float s = sc_cur[0];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[c + i] = fmaf(s, v0[i], acc[c + i]);
+            if (c + 16 < C::kCols) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) acc[c + 16 + i] = fmaf(s, v1[i], acc[c + 16 + i]);
+            }
+          } else {
+            const float scv = sc_cur[c / 32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              acc[c + i] = fmaf(__shfl_sync(0xffffffffu, scv, i), v0[i], acc[c + i]);
+            if (c + 16 < C::kCols) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[c + 16 + i] =
+                    fmaf(__shfl_sync(0xffffffffu, scv, 16 + i), v1[i], acc[c + 16 + i]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        tb ^= 1;
+        if (tb == 0) tphase ^= 1u;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) sc_cur[c] = sc_next[c];
+      }
+      if (!ok) break;
+
+      if (args.splits == 1) {
+        if constexpr (!kSwap) {
+          // row m of Y, columns [n0, n0 + kCols): 16-byte stores of 8 bf16
+          const int n0 = ct * BN + col0;
+          if (m < args.M) {
+            __nv_bfloat16* yrow = args.y + static_cast<int64_t>(m) * args.N;
+#pragma unroll
+            for (int c = 0; c < C::kCols; c += 8) {
+              if (n0 + c < args.N) {
+                uint4 pk;
+                pk.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
+                pk.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+                pk.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+                pk.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+                *reinterpret_cast<uint4*>(yrow + n0 + c) = pk;
+              }
+            }
+          }
+        } else {
+          // column j of the tile is token ct*BN + col0 + j; row is weight row n
+          const int n = rt * 128 + row;
+          if (n < args.N) {
+#pragma unroll
+            for (int j = 0; j < C::kCols; ++j) {
+              const int tok = ct * BN + col0 + j;
+              if (tok < args.M)
+                args.y[static_cast<int64_t>(tok) * args.N + n] = __float2bfloat16_rn(acc[j]);
+            }
+          }
+        }
+      }
+    }
+    if (!ok) {
+      record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+
+  if (args.splits > 1) {
+    // ---------------------------------------- split-K reduction in the cluster --
+    // Each CTA publishes its fp32 partial tile [BN][128] (column-major in the
+    // MMA's row index) in its own (drained) stage memory; rank r then sums
+    // columns [r*BN/S, (r+1)*BN/S) over ranks 0..S-1 in order and writes Y.
+    float* red = reinterpret_cast<float*>(smem);
+    if (warp >= 4) {
+      const int wg = (warp - 4) >> 2;
+      const int row = (warp & 3) * 32 + lane;
+#pragma unroll
+      for (int j = 0; j < C::kCols; ++j) red[(wg * C::kCols + j) * 128 + row] = acc[j];
+    }
+    __syncwarp();
+    cluster_sync();
+    int last_rt, last_ct;  // split-K CTAs own exactly one tile: blockIdx.y
+    tile_coords(blockIdx.y, args.row_tiles, args.col_tiles, last_rt, last_ct);
+    if (!*abort_flag) {
+      const int S = args.splits;
+      const int rank = static_cast<int>(cluster_ctarank());
+      const int j_lo = rank * BN / S, j_hi = (rank + 1) * BN / S;
+      const int total4 = (j_hi - j_lo) * 32;
+      for (int idx = threadIdx.x; idx < total4; idx += C::kThreads) {
+        const int j = j_lo + idx / 32;
+        const int r4 = (idx % 32) * 4;
+        const uint32_t local = smem_u32(red + j * 128 + r4);
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < S; ++q) {
+          const float4 v = ld_cluster_f32x4(map_cluster(local, static_cast<uint32_t>(q)));
+          s.x += v.x;
+          s.y += v.y;
+          s.z += v.z;
+          s.w += v.w;
+        }
+        int out_row, out_col;  // Y coordinates of element (j, r4)
+        if constexpr (kSwap) {
+          out_row = last_ct * BN + j;
+          out_col = last_rt * 128 + r4;
+        } else {
+          out_row = last_rt * 128 + r4;  // (prefill split-K is not used)
+          out_col = last_ct * BN + j;
+        }
+        if (kSwap && out_row < args.M && out_col < args.N) {
+          uint2 pk;
+          pk.x = pack_bf16x2(s.x, s.y);
+          pk.y = pack_bf16x2(s.z, s.w);
+          *reinterpret_cast<uint2*>(args.y + static_cast<int64_t>(out_row) * args.N + out_col) =
+              pk;
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync();
+  }
+
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side --
+
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
+int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
+               const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
+  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG>;
+  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG>;
+  static std::once_flag flags[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8BS_ERR_CUDA;
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(flags[dev], [&] {
+    attr_err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return FP8BS_ERR_CUDA;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(grid_y), 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  cfg.numAttrs = 0;
+  if (splits > 1) {
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = static_cast<unsigned>(splits);
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, te, a) != cudaSuccess) return FP8BS_ERR_CUDA;
+  return FP8BS_OK;
+}
+
+inline int next_pow2_at_least16(int64_t v) {
+  int b = 16;
+  while (b < v) b <<= 1;
+  return b;
+}
+
+// K split of a swapped (weights-on-M) launch: spread `tiles` units over the
+// SMs with a cluster of up to 8 CTAs per tile when the tiles alone do not
+// fill the GPU; at least one K-block per split.
+inline int choose_splits(int tiles, int sm_count, int KB) {
+  int S = 1;
+  if (tiles < sm_count) {
+    S = sm_count / tiles;
+    if (S > 8) S = 8;
+    if (S > KB) S = KB;
+    if (S < 1) S = 1;
+  }
+  return S;
+}
+
+}  // namespace gemm_detail
+
+}  // namespace fp8bs

@@ -37,9 +37,11 @@ struct DeviceInfo {
 };
 int current_device_info(DeviceInfo* info);
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// cuTensorMapEncodeTiled through the runtime's driver entry point: a 2-D
+// tensor of bytes, `inner` contiguous x `outer` rows `row_stride_bytes` apart.
+enum TmapSwizzle { kSwizzleNone = 0, kSwizzle64B = 64, kSwizzle128B = 128 };
 int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                      int swizzle_128b);
+                      TmapSwizzle swizzle);
 
 }  // namespace fp8bs

@@ -33,6 +33,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -165,10 +166,13 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.out = None
+        self._own_file = None   # the temporary file this sampler created
 
     def __enter__(self):
         try:
-            self.out = open(os.devnull if False else "/tmp/fp8bs_clocks_%d.csv" % os.getpid(), "w+")
+            fd, path = tempfile.mkstemp(prefix="fp8bs_clocks_", suffix=".csv")
+            self._own_file = path
+            self.out = os.fdopen(fd, "w+")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "200"],
@@ -192,12 +196,13 @@ class ClockSampler:
         self.out.flush()
         self.out.seek(0)
         rows = [l.strip().split(", ") for l in self.out.read().splitlines() if l.strip()]
-        name = self.out.name
         self.out.close()
-        try:
-            os.remove(name)
-        except OSError:
-            pass
+        if self._own_file is not None:
+            try:
+                os.remove(self._own_file)
+            except OSError:
+                pass
+            self._own_file = None
         sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for r in rows:

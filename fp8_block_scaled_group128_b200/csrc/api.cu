@@ -71,16 +71,17 @@ int current_device_info(DeviceInfo* info) {
   return FP8BS_OK;
 }
 
-int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
-                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                      TmapSwizzle swizzle) {
+int encode_tmap_2d(void* map_out, const void* base, int elem_bytes, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                   uint32_t box_outer, TmapSwizzle swizzle) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return FP8BS_ERR_CUDA;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(static_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+  const CUresult r = fn(static_cast<CUtensorMap*>(map_out),
+                        elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                         const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
                         swizzle == kSwizzle128B  ? CU_TENSOR_MAP_SWIZZLE_128B

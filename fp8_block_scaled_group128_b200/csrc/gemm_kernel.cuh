@@ -74,9 +74,12 @@ struct Cfg {
   static constexpr int kThreads = 128 * (1 + kEpiWG);
   static constexpr int kCols = BN / kEpiWG;  // accumulator columns per epilogue thread
   static_assert(kCols % 16 == 0 && kCols <= 128, "epilogue column split");
-  // TMEM: two partial buffers of BN columns, then (sparse) two metadata
-  // buffers of 4 columns; the allocation is a power of two >= 32.
-  static constexpr int kTmemUsed = 2 * BN + (kSparse ? 8 : 0);
+  // TMEM: kBufs partial buffers of BN columns (up to 8, so the MMA can run
+  // ahead of the promotion), then (sparse) two metadata buffers of 4
+  // columns; the allocation is a power of two >= 32.
+  static constexpr int kBufs = (512 - (kSparse ? 8 : 0)) / BN < 8 ? (512 - (kSparse ? 8 : 0)) / BN : 8;
+  static_assert(kBufs >= 2, "at least two TMEM partial buffers");
+  static constexpr int kTmemUsed = kBufs * BN + (kSparse ? 8 : 0);
   static constexpr int kTmemCols =
       kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
   static_assert(kTmemUsed <= 512, "TMEM has 512 columns");
@@ -85,7 +88,7 @@ struct Cfg {
   static constexpr int kOffB = kStages * kABytes;
   static constexpr int kOffE = kOffB + kStages * kBBytes;
   static constexpr int kOffBar = kOffE + (kSparse ? kStages * kEBytes : 0);
-  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kNumBars = 2 * kStages + 2 * kBufs + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
   static constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + slack to align the base
@@ -127,8 +130,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* mma_done = tempty + 2;
+  uint64_t* tempty = tfull + C::kBufs;
+  uint64_t* mma_done = tempty + C::kBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
 
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kBufs; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 4 * kEpiWG);
     }
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
             // metadata of this K-block -> TMEM (4 columns, lane = weight row),
             // then two sparse MMAs of logical depth 64 (32 compressed bytes
             // of A and 64 bytes of B each), reading 2 metadata columns each
-            const uint32_t te = tmem_base + static_cast<uint32_t>(2 * BN) + 4u * e_buf;
+            const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
             e_buf ^= 1u;
             tmem_cp_128x128b(te, noswizzle_kmajor_desc(smem_u32(sm_e + stage * kEBytes), 128));
 #pragma unroll
@@ -276,8 +279,10 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
             stage = 0;
             phase ^= 1u;
           }
-          tb ^= 1;
-          if (tb == 0) tphase ^= 1u;
+          if (++tb == C::kBufs) {
+            tb = 0;
+            tphase ^= 1u;
+          }
         }
       }
       if (!ok) {
@@ -317,64 +322,78 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) tok_l[c] = ct * BN + col0 + 32 * c + lane;
 
-      auto load_scales = [&](int kb, float* sc) {
+      // The loads land in the ring untouched (the product is formed only when
+      // the K-block is consumed, so nothing waits on a load early).
+      auto load_scales = [&](int kb, float* sa_v, float& sw_v) {
         if constexpr (!kSwap) {
-          sc[0] = row_ok ? sa_row[kb] * args.sw[static_cast<int64_t>(nb) * KB + kb] : 0.0f;
+          sa_v[0] = row_ok ? sa_row[kb] : 0.0f;
+          sw_v = row_ok ? args.sw[static_cast<int64_t>(nb) * KB + kb] : 0.0f;
         } else {
-          const float swv = args.sw[static_cast<int64_t>(rt) * KB + kb];
+          sw_v = args.sw[static_cast<int64_t>(rt) * KB + kb];
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
             const bool tok_ok = tok_l[c] < args.M && (32 * c + lane) < C::kCols;
-            sc[c] = tok_ok ? swv * args.sa[static_cast<int64_t>(tok_l[c]) * KB + kb] : 0.0f;
+            sa_v[c] = tok_ok ? args.sa[static_cast<int64_t>(tok_l[c]) * KB + kb] : 0.0f;
           }
         }
       };
-      float sc_cur[kChunks], sc_next[kChunks];
-      if (kb0 < kb1) load_scales(kb0, sc_cur);
+      // Scales are prefetched kPrefetch K-blocks ahead into a register ring
+      // indexed at compile time (the K loop is unrolled by kPrefetch).
+      constexpr int kPrefetch = 4;
+      float ring_a[kPrefetch][kChunks];
+      float ring_w[kPrefetch];
+#pragma unroll
+      for (int d = 0; d < kPrefetch; ++d)
+        if (kb0 + d < kb1) load_scales(kb0 + d, ring_a[d], ring_w[d]);
 
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (kb + 1 < kb1) load_scales(kb + 1, sc_next);
-        if (!mbar_wait(&tfull[tb], tphase, limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
+      for (int kb_base = kb0; ok && kb_base < kb1; kb_base += kPrefetch) {
 #pragma unroll
-        for (int c = 0; c < C::kCols; c += 32) {
-          float v0[16], v1[16];
-          tmem_ld16(taddr + c, v0);
-          if (c + 16 < C::kCols) tmem_ld16(taddr + c + 16, v1);
-          tmem_wait_ld();
-          if constexpr (!kSwap) {
-            const float s = sc_cur[0];
+        for (int d = 0; d < kPrefetch; ++d) {
+          const int kb = kb_base + d;
+          if (!ok || kb >= kb1) break;
+          if (!mbar_wait(&tfull[tb], tphase, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[c + i] = fmaf(s, v0[i], acc[c + i]);
-            if (c + 16 < C::kCols) {
+          for (int c = 0; c < C::kCols; c += 32) {
+            float v0[16], v1[16];
+            tmem_ld16(taddr + c, v0);
+            if (c + 16 < C::kCols) tmem_ld16(taddr + c + 16, v1);
+            tmem_wait_ld();
+            if constexpr (!kSwap) {
+              const float sc = ring_a[d][0] * ring_w[d];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) acc[c + 16 + i] = fmaf(s, v1[i], acc[c + 16 + i]);
-            }
-          } else {
-            const float scv = sc_cur[c / 32];
+              for (int i = 0; i < 16; ++i) acc[c + i] = fmaf(sc, v0[i], acc[c + i]);
+              if (c + 16 < C::kCols) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[c + i] = fmaf(__shfl_sync(0xffffffffu, scv, i), v0[i], acc[c + i]);
-            if (c + 16 < C::kCols) {
+                for (int i = 0; i < 16; ++i) acc[c + 16 + i] = fmaf(sc, v1[i], acc[c + 16 + i]);
+              }
+            } else {
+              const float scv = ring_w[d] * ring_a[d][c / 32];
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                acc[c + 16 + i] =
-                    fmaf(__shfl_sync(0xffffffffu, scv, 16 + i), v1[i], acc[c + 16 + i]);
+                acc[c + i] = fmaf(__shfl_sync(0xffffffffu, scv, i), v0[i], acc[c + i]);
+              if (c + 16 < C::kCols) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  acc[c + 16 + i] =
+                      fmaf(__shfl_sync(0xffffffffu, scv, 16 + i), v1[i], acc[c + 16 + i]);
+              }
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);
+          if (++tb == C::kBufs) {
+            tb = 0;
+            tphase ^= 1u;
+          }
+          if (kb + kPrefetch < kb1) load_scales(kb + kPrefetch, ring_a[d], ring_w[d]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[tb]);
-        tb ^= 1;
-        if (tb == 0) tphase ^= 1u;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) sc_cur[c] = sc_next[c];
       }
       if (!ok) break;
 

@@ -40,8 +40,17 @@ int current_device_info(DeviceInfo* info);
 // cuTensorMapEncodeTiled through the runtime's driver entry point: a 2-D
 // tensor of bytes, `inner` contiguous x `outer` rows `row_stride_bytes` apart.
 enum TmapSwizzle { kSwizzleNone = 0, kSwizzle64B = 64, kSwizzle128B = 128 };
-int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
-                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                      TmapSwizzle swizzle);
+int encode_tmap_2d(void* map_out, const void* base, int elem_bytes, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                   uint32_t box_outer, TmapSwizzle swizzle);
+inline int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, uint64_t outer,
+                             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                             TmapSwizzle swizzle) {
+  return encode_tmap_2d(map_out, base, 1, inner, outer, row_stride_bytes, box_inner, box_outer,
+                        swizzle);
+}
+
+// Current bound of the kernels' mbarrier waits (SM cycles).
+long long wait_limit();
 
 }  // namespace fp8bs

@@ -91,6 +91,25 @@ int encode_tmap_2d(void* map_out, const void* base, int elem_bytes, uint64_t inn
   return r == CUDA_SUCCESS ? FP8BS_OK : FP8BS_ERR_CUDA;
 }
 
+int encode_tmap_kblocks(void* map_out, const void* base, uint64_t block_bytes, uint64_t rows,
+                        uint64_t n_blocks, uint64_t row_stride_bytes, uint32_t box_rows,
+                        uint32_t box_blocks, TmapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return FP8BS_ERR_CUDA;
+  const cuuint64_t dims[3] = {block_bytes, rows, n_blocks};
+  const cuuint64_t strides[2] = {row_stride_bytes, block_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(block_bytes), box_rows, box_blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                        const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle == kSwizzle128B  ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle == kSwizzle64B ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8BS_OK : FP8BS_ERR_CUDA;
+}
+
 long long wait_limit() { return g_wait_limit.load(); }
 
 int* device_error_word() {

@@ -24,23 +24,26 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   a.err = err;
   alignas(64) CUtensorMap ta, tb;
 
+  const uint64_t KB = static_cast<uint64_t>(K / 128);
   if (M <= 256) {
-    // Decode: weights on the MMA M side, tokens on the MMA N side.
+    // Decode: weights on the MMA M side, tokens on the MMA N side; stages of
+    // two K-blocks.
+    constexpr int kKS = 2;
     const int BN = next_pow2_at_least16(M);
     a.row_tiles = static_cast<int>((N + 127) / 128);
     a.col_tiles = 1;
     const int tiles = a.row_tiles;
-    const int S = choose_splits(tiles, dev.sm_count, a.KB);
+    const int S = choose_splits(tiles, dev.sm_count, a.KB, kKS);
     a.splits = S;
     const int grid_y = S > 1 ? tiles : (tiles < dev.sm_count ? tiles : dev.sm_count);
-    if (int st = encode_tmap_2d_u8(&ta, qw, K, N, K, 128, 128, kSwizzle128B)) return st;
-    if (int st = encode_tmap_2d_u8(&tb, qa, K, M, K, 128, BN, kSwizzle128B)) return st;
+    if (int st = encode_tmap_kblocks(&ta, qw, 128, N, KB, K, 128, kKS, kSwizzle128B)) return st;
+    if (int st = encode_tmap_kblocks(&tb, qa, 128, M, KB, K, BN, kKS, kSwizzle128B)) return st;
     switch (BN) {
-      case 16: return launch_cfg<16, true, false, 11, 1>(ta, tb, ta, a, grid_y, S, stream);
-      case 32: return launch_cfg<32, true, false, 10, 1>(ta, tb, ta, a, grid_y, S, stream);
-      case 64: return launch_cfg<64, true, false, 8, 1>(ta, tb, ta, a, grid_y, S, stream);
-      case 128: return launch_cfg<128, true, false, 6, 2>(ta, tb, ta, a, grid_y, S, stream);
-      default: return launch_cfg<256, true, false, 4, 2>(ta, tb, ta, a, grid_y, S, stream);
+      case 16: return launch_cfg<16, true, false, 5, 1, kKS>(ta, tb, ta, a, grid_y, S, stream);
+      case 32: return launch_cfg<32, true, false, 5, 1, kKS>(ta, tb, ta, a, grid_y, S, stream);
+      case 64: return launch_cfg<64, true, false, 4, 1, kKS>(ta, tb, ta, a, grid_y, S, stream);
+      case 128: return launch_cfg<128, true, false, 3, 2, kKS>(ta, tb, ta, a, grid_y, S, stream);
+      default: return launch_cfg<256, true, false, 2, 2, kKS>(ta, tb, ta, a, grid_y, S, stream);
     }
   }
   // Prefill: tokens on the MMA M side, 256 weight rows on the MMA N side.
@@ -51,9 +54,9 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
   if (tiles > 0x7FFFFFFF) return FP8BS_ERR_SHAPE;
   const int grid_y = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  if (int st = encode_tmap_2d_u8(&ta, qa, K, M, K, 128, 128, kSwizzle128B)) return st;
-  if (int st = encode_tmap_2d_u8(&tb, qw, K, N, K, 128, BN, kSwizzle128B)) return st;
-  return launch_cfg<BN, false, false, 4, 2>(ta, tb, ta, a, grid_y, 1, stream);
+  if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, 128, 1, kSwizzle128B)) return st;
+  if (int st = encode_tmap_kblocks(&tb, qw, 128, N, KB, K, BN, 1, kSwizzle128B)) return st;
+  return launch_cfg<BN, false, false, 4, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
 }
 
 }  // namespace fp8bs

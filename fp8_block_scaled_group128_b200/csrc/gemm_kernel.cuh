@@ -61,16 +61,21 @@ struct GemmArgs {
   int* err;             // device error word
 };
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
 struct Cfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
   static_assert((BN & (BN - 1)) == 0, "BN is a power of two (TMEM allocation)");
   static_assert(!kSparse || kSwap, "the 2:4 operand is the weight, on the MMA M side");
-  // A stage: 128 rows x 128 B (dense, 128 B swizzle) or 128 rows x 64 B of
-  // compressed 2:4 values (64 B swizzle); B stage: BN rows x 128 B.
-  static constexpr int kABytes = kSparse ? 128 * kBK / 2 : 128 * kBK;
-  static constexpr int kBBytes = BN * kBK;
-  static constexpr int kStageBytes = kABytes + kBBytes + (kSparse ? kEBytes : 0);
+  // A stage holds kKS K-blocks (one 3-D TMA box per operand, so each copy is
+  // large): A: kKS x 128 rows x 128 B (dense, 128 B swizzle) or kKS x 128 rows
+  // x 64 B of compressed 2:4 values (64 B swizzle); B: kKS x BN rows x 128 B;
+  // sparse metadata: kKS x 128 rows x 16 B.
+  static constexpr int kAKb = kSparse ? 128 * kBK / 2 : 128 * kBK;  // A bytes per K-block
+  static constexpr int kBKb = BN * kBK;                             // B bytes per K-block
+  static constexpr int kABytes = kKS * kAKb;
+  static constexpr int kBBytes = kKS * kBKb;
+  static constexpr int kEStage = kSparse ? kKS * kEBytes : 0;
+  static constexpr int kStageBytes = kABytes + kBBytes + kEStage;
   static constexpr int kThreads = 128 * (1 + kEpiWG);
   static constexpr int kCols = BN / kEpiWG;  // accumulator columns per epilogue thread
   static_assert(kCols % 16 == 0 && kCols <= 128, "epilogue column split");
@@ -87,7 +92,7 @@ struct Cfg {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kStages * kABytes;
   static constexpr int kOffE = kOffB + kStages * kBBytes;
-  static constexpr int kOffBar = kOffE + (kSparse ? kStages * kEBytes : 0);
+  static constexpr int kOffBar = kOffE + kStages * kEStage;
   static constexpr int kNumBars = 2 * kStages + 2 * kBufs + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
@@ -95,7 +100,7 @@ struct Cfg {
   // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
   static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-  static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage buffers stay 1024-aligned");
+  static_assert(kAKb % 1024 == 0 && kBKb % 1024 == 0, "stage buffers stay 1024-aligned");
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int row_tiles, int col_tiles, int& rt,
@@ -114,12 +119,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
-__global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThreads, 1)
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
+__global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>::kThreads, 1)
     block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_e, const GemmArgs args) {
-  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG>;
+  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   constexpr int kABytes = C::kABytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -138,8 +143,14 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x;
-  const int kb0 = static_cast<int>(static_cast<long long>(split) * args.KB / args.splits);
-  const int kb1 = static_cast<int>(static_cast<long long>(split + 1) * args.KB / args.splits);
+  // K range of this split, boundaries rounded to whole stages (kKS K-blocks)
+  const int kb0 = split == 0 ? 0
+                             : static_cast<int>(static_cast<long long>(split) * args.KB /
+                                                args.splits) / kKS * kKS;
+  const int kb1 = split == args.splits - 1
+                      ? args.KB
+                      : static_cast<int>(static_cast<long long>(split + 1) * args.KB /
+                                         args.splits) / kKS * kKS;
   const int num_tiles = args.row_tiles * args.col_tiles;
   const long long limit = args.wait_limit;
 
@@ -174,42 +185,25 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer --
-      uint64_t pol_a = 0, pol_b = 0;
-      if constexpr (kSwap) {
-        pol_a = policy_evict_first();
-        pol_b = policy_evict_last();
-      }
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       for (int tile = blockIdx.y; tile < num_tiles && !*abort_flag; tile += gridDim.y) {
         int rt, ct;
         tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += kKS) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
             record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
             *abort_flag = 1;
             break;
           }
+          // one box per operand covers K-blocks [kb, kb + kKS) (K-blocks past
+          // the end of K read as zero and are not used)
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          if constexpr (kSparse) {
-            // compressed values: 64 B per row per K-block; metadata: 16 B per row
-            tma_load_2d_hint(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * (kBK / 2),
-                             rt * 128, pol_a);
-            tma_load_2d_hint(sm_e + stage * kEBytes, &tmap_e, &full[stage], kb * 16, rt * 128,
-                             pol_a);
-            tma_load_2d_hint(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK,
-                             ct * BN, pol_b);
-          } else if constexpr (kSwap) {
-            // decode: weights are streamed once, activations are shared by all CTAs
-            tma_load_2d_hint(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * kBK, rt * 128,
-                             pol_a);
-            tma_load_2d_hint(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK,
-                             ct * BN, pol_b);
-          } else {
-            tma_load_2d(sm_a + stage * kABytes, &tmap_a, &full[stage], kb * kBK, rt * 128);
-            tma_load_2d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], kb * kBK, ct * BN);
-          }
+          tma_load_3d(sm_a + stage * C::kABytes, &tmap_a, &full[stage], 0, rt * 128, kb);
+          if constexpr (kSparse)
+            tma_load_3d(sm_e + stage * C::kEStage, &tmap_e, &full[stage], 0, rt * 128, kb);
+          tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, ct * BN, kb);
           ++issued;
           if (++stage == kStages) {
             stage = 0;
@@ -240,48 +234,54 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
       uint32_t e_buf = 0;  // sparse: TMEM metadata buffer, alternating per K-block
       bool ok = true;
       for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        for (int kb = kb0; ok && kb < kb1; kb += kKS) {
           if (!mbar_wait(&full[stage], phase, limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
-          const uint32_t a0 = smem_u32(sm_a + stage * kABytes);
-          const uint32_t b0 = smem_u32(sm_b + stage * C::kBBytes);
-          if constexpr (kSparse) {
-            // metadata of this K-block -> TMEM (4 columns, lane = weight row),
-            // then two sparse MMAs of logical depth 64 (32 compressed bytes
-            // of A and 64 bytes of B each), reading 2 metadata columns each
-            const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
-            e_buf ^= 1u;
-            tmem_cp_128x128b(te, noswizzle_kmajor_desc(smem_u32(sm_e + stage * kEBytes), 128));
 #pragma unroll
-            for (int k = 0; k < kBK / 64; ++k) {
-              mma_sp_f8f6f4(d, sw64_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 64 * k),
-                            te + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
+          for (int j = 0; j < kKS; ++j) {
+            if (kb + j >= kb1) break;
+            if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
+              ok = false;
+              break;
             }
-          } else {
+            tc_fence_after();
+            const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
+            const uint32_t a0 = smem_u32(sm_a + stage * C::kABytes + j * C::kAKb);
+            const uint32_t b0 = smem_u32(sm_b + stage * C::kBBytes + j * C::kBKb);
+            if constexpr (kSparse) {
+              // metadata of this K-block -> TMEM (4 columns, lane = weight
+              // row), then two sparse MMAs of logical depth 64 (32 compressed
+              // bytes of A and 64 bytes of B each), reading 2 metadata columns
+              const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
+              e_buf ^= 1u;
+              tmem_cp_128x128b(
+                  te, noswizzle_kmajor_desc(smem_u32(sm_e + stage * C::kEStage + j * kEBytes), 128));
 #pragma unroll
-            for (int k = 0; k < kBK / 32; ++k) {
-              mma_f8f6f4(d, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
-                         C::kIdesc, k > 0 ? 1u : 0u);
+              for (int k = 0; k < kBK / 64; ++k) {
+                mma_sp_f8f6f4(d, sw64_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 64 * k),
+                              te + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < kBK / 32; ++k) {
+                mma_f8f6f4(d, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
+                           C::kIdesc, k > 0 ? 1u : 0u);
+              }
+            }
+            mma_commit(&tfull[tb]);
+            if (++tb == C::kBufs) {
+              tb = 0;
+              tphase ^= 1u;
             }
           }
+          // the stage is free once every MMA that reads it has completed
           mma_commit(&empty[stage]);
-          mma_commit(&tfull[tb]);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
-          }
-          if (++tb == C::kBufs) {
-            tb = 0;
-            tphase ^= 1u;
           }
         }
       }
@@ -501,11 +501,11 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG>::kThr
 
 // ------------------------------------------------------------------ host side --
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
                const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
-  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG>;
-  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG>;
+  using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
+  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   static std::once_flag flags[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8BS_ERR_CUDA;
@@ -544,12 +544,12 @@ inline int next_pow2_at_least16(int64_t v) {
 // K split of a swapped (weights-on-M) launch: spread `tiles` units over the
 // SMs with a cluster of up to 8 CTAs per tile when the tiles alone do not
 // fill the GPU; at least one K-block per split.
-inline int choose_splits(int tiles, int sm_count, int KB) {
+inline int choose_splits(int tiles, int sm_count, int KB, int ks) {
   int S = 1;
   if (tiles < sm_count) {
     S = sm_count / tiles;
     if (S > 8) S = 8;
-    if (S > KB) S = KB;
+    if (S > KB / ks) S = KB / ks;
     if (S < 1) S = 1;
   }
   return S;

@@ -32,24 +32,26 @@ int launch_sparse24_gemm(const void* qa, const float* sa, const void* vals, cons
   a.err = err;
 
   const int BN = M <= 128 ? next_pow2_at_least16(M) : 128;
+  const int kKS = BN <= 32 ? 4 : 2;   // K-blocks per stage (bigger TMA copies)
   a.row_tiles = static_cast<int>((N + 127) / 128);
   a.col_tiles = static_cast<int>((M + BN - 1) / BN);
   const int64_t tiles64 = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
   if (tiles64 > 65535LL * 148) return FP8BS_ERR_SHAPE;
   const int tiles = static_cast<int>(tiles64);
-  const int S = choose_splits(tiles, dev.sm_count, a.KB);
+  const int S = choose_splits(tiles, dev.sm_count, a.KB, kKS);
   a.splits = S;
   const int grid_y = S > 1 ? tiles : (tiles < dev.sm_count ? tiles : dev.sm_count);
 
+  const uint64_t KB = static_cast<uint64_t>(K / 128);
   alignas(64) CUtensorMap ta, tb, te;
-  if (int st = encode_tmap_2d_u8(&ta, vals, K / 2, N, K / 2, 64, 128, kSwizzle64B)) return st;
-  if (int st = encode_tmap_2d_u8(&te, meta, K / 8, N, K / 8, 16, 128, kSwizzleNone)) return st;
-  if (int st = encode_tmap_2d_u8(&tb, qa, K, M, K, 128, BN, kSwizzle128B)) return st;
+  if (int st = encode_tmap_kblocks(&ta, vals, 64, N, KB, K / 2, 128, kKS, kSwizzle64B)) return st;
+  if (int st = encode_tmap_kblocks(&te, meta, 16, N, KB, K / 8, 128, kKS, kSwizzleNone)) return st;
+  if (int st = encode_tmap_kblocks(&tb, qa, 128, M, KB, K, BN, kKS, kSwizzle128B)) return st;
   switch (BN) {
-    case 16: return launch_cfg<16, true, true, 16, 1>(ta, tb, te, a, grid_y, S, stream);
-    case 32: return launch_cfg<32, true, true, 14, 1>(ta, tb, te, a, grid_y, S, stream);
-    case 64: return launch_cfg<64, true, true, 11, 1>(ta, tb, te, a, grid_y, S, stream);
-    default: return launch_cfg<128, true, true, 7, 2>(ta, tb, te, a, grid_y, S, stream);
+    case 16: return launch_cfg<16, true, true, 4, 1, 4>(ta, tb, te, a, grid_y, S, stream);
+    case 32: return launch_cfg<32, true, true, 3, 1, 4>(ta, tb, te, a, grid_y, S, stream);
+    case 64: return launch_cfg<64, true, true, 5, 1, 2>(ta, tb, te, a, grid_y, S, stream);
+    default: return launch_cfg<128, true, true, 3, 2, 2>(ta, tb, te, a, grid_y, S, stream);
   }
 }
 

@@ -50,6 +50,15 @@ inline int encode_tmap_2d_u8(void* map_out, const void* base, uint64_t inner, ui
                         swizzle);
 }
 
+// A 3-D view of a row-major byte matrix [rows][row_stride_bytes] cut into
+// K-blocks: dim 0 = `block_bytes` contiguous bytes of one K-block, dim 1 = the
+// rows (`row_stride_bytes` apart), dim 2 = the K-blocks (`block_bytes` apart).
+// A box {block_bytes, box_rows, box_blocks} lands in shared memory as
+// box_blocks slabs of [box_rows][block_bytes].
+int encode_tmap_kblocks(void* map_out, const void* base, uint64_t block_bytes, uint64_t rows,
+                        uint64_t n_blocks, uint64_t row_stride_bytes, uint32_t box_rows,
+                        uint32_t box_blocks, TmapSwizzle swizzle);
+
 // Current bound of the kernels' mbarrier waits (SM cycles).
 long long wait_limit();
 

@@ -46,52 +46,52 @@ struct QArgs {
   int* err;
 };
 
-// Kept pair of a group of 4 bf16 magnitudes (sign cleared): rank each member
-// by how many others beat it (larger magnitude, or equal magnitude at a lower
-// index); ranks 0 and 1 are kept. Returns the nibble i0 | i1 << 2, i0 < i1.
-__device__ __forceinline__ uint32_t select24(const uint32_t (&mag)[4]) {
-  uint32_t keep = 0;
+// 2:4 selection of one group of 4 bf16 values held in a 64-bit word (value j
+// in bits 16j..16j+15). Each member gets the key (|w| bits << 2) | (3 - j):
+// a larger magnitude wins, and equal magnitudes go to the lower index. The two
+// largest keys (a 4-input max / second-max network) are the kept pair.
+// Returns i0 | i1 << 2 (i0 < i1) and the two kept bf16 patterns in position
+// order.
+__device__ __forceinline__ uint32_t select24(uint64_t g, uint32_t& k0, uint32_t& k1) {
+  uint32_t key[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int beaten = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j == i) continue;
-      beaten += (mag[j] > mag[i]) || (mag[j] == mag[i] && j < i);
-    }
-    keep |= (beaten < 2 ? 1u : 0u) << i;
-  }
-  const uint32_t i0 = __ffs(keep) - 1;   // lowest kept position
-  const uint32_t i1 = 31 - __clz(keep);  // highest kept position
+  for (int j = 0; j < 4; ++j)
+    key[j] = ((static_cast<uint32_t>(g >> (16 * j)) & 0x7FFFu) << 2) | static_cast<uint32_t>(3 - j);
+  const uint32_t a = max(key[0], key[1]), b = min(key[0], key[1]);
+  const uint32_t c = max(key[2], key[3]), d = min(key[2], key[3]);
+  const uint32_t top1 = max(a, c);
+  const uint32_t top2 = max(min(a, c), max(b, d));
+  const uint32_t p1 = 3u - (top1 & 3u), p2 = 3u - (top2 & 3u);
+  const uint32_t i0 = min(p1, p2), i1 = max(p1, p2);
+  k0 = static_cast<uint32_t>(g >> (16 * i0)) & 0xFFFFu;
+  k1 = static_cast<uint32_t>(g >> (16 * i1)) & 0xFFFFu;
   return i0 | (i1 << 2);
 }
 
-// 2:4 selection and encoding of the 8 weights of one thread-row: returns the
-// 4 value bytes, sets the metadata byte and the pruned bf16 words.
+// 2:4 selection and encoding of the 8 weights (two groups) of one thread-row:
+// returns the 4 value bytes, sets the metadata byte and the pruned bf16 words.
 __device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d, uint32_t& nib2,
                                            uint4& pruned) {
-  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
-  uint32_t packed = 0, pr[4] = {0u, 0u, 0u, 0u};
-  nib2 = 0;
-#pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const uint32_t e[4] = {words[2 * g] & 0xFFFFu, words[2 * g] >> 16, words[2 * g + 1] & 0xFFFFu,
-                           words[2 * g + 1] >> 16};
-    const uint32_t mag[4] = {e[0] & 0x7FFFu, e[1] & 0x7FFFu, e[2] & 0x7FFFu, e[3] & 0x7FFFu};
-    const uint32_t nib = select24(mag);
-    const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-    uint32_t k0 = 0, k1 = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const bool is0 = j == static_cast<int>(i0), is1 = j == static_cast<int>(i1);
-      if (is0) k0 = e[j];
-      if (is1) k1 = e[j];
-      pr[2 * g + (j >> 1)] |= ((is0 || is1) ? e[j] : 0u) << (16 * (j & 1));
-    }
-    packed |= (e4m3_code_bf16(d, k0) | (e4m3_code_bf16(d, k1) << 8)) << (16 * g);
-    nib2 |= nib << (4 * g);
+  const uint64_t g0 = (static_cast<uint64_t>(v.y) << 32) | v.x;
+  const uint64_t g1 = (static_cast<uint64_t>(v.w) << 32) | v.z;
+  uint32_t a0, a1, b0, b1;
+  const uint32_t n0 = select24(g0, a0, a1);
+  const uint32_t n1 = select24(g1, b0, b1);
+  nib2 = n0 | (n1 << 4);
+  uint32_t packed;
+  if (d.s == 0.0f) {
+    packed = ((a0 & 0x8000u) ? 0x80u : 0u) | ((a1 & 0x8000u) ? 0x8000u : 0u) |
+             ((b0 & 0x8000u) ? 0x800000u : 0u) | ((b1 & 0x8000u) ? 0x80000000u : 0u);
+  } else {
+    packed = e4m3x2(d, __uint_as_float(a0 << 16), __uint_as_float(a1 << 16)) |
+             (e4m3x2(d, __uint_as_float(b0 << 16), __uint_as_float(b1 << 16)) << 16);
   }
-  pruned = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+  // pruned weights: keep positions i0, i1 of each group, +0 elsewhere
+  const uint64_t m0 = (0xFFFFull << (16 * (n0 & 3u))) | (0xFFFFull << (16 * (n0 >> 2)));
+  const uint64_t m1 = (0xFFFFull << (16 * (n1 & 3u))) | (0xFFFFull << (16 * (n1 >> 2)));
+  const uint64_t p0 = g0 & m0, p1 = g1 & m1;
+  pruned = make_uint4(static_cast<uint32_t>(p0), static_cast<uint32_t>(p0 >> 32),
+                      static_cast<uint32_t>(p1), static_cast<uint32_t>(p1 >> 32));
   return packed;
 }
 

@@ -96,7 +96,10 @@ struct Cfg {
   static constexpr int kNumBars = 2 * kStages + 2 * kBufs + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
-  static constexpr int kSmemBytes = kOffAbort + 4 + 1024;  // + slack to align the base
+  // decode: per-epilogue-warp column scales of the current K-block
+  static constexpr int kOffScr = (kOffAbort + 4 + 15) / 16 * 16;
+  static constexpr int kScrBytes = kSwap ? 4 * kEpiWG * kCols * 4 : 0;
+  static constexpr int kSmemBytes = kOffScr + kScrBytes + 1024;  // + slack to align the base
   // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
   static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -178,6 +181,10 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up above touches no global memory; inputs may come from the previous
+  // kernel of the stream.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   // Registers of the epilogue threads that outlive the role loop (split-K).
   float acc[C::kCols];
@@ -300,6 +307,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     const int row = quarter * 32 + lane;
     const int col0 = wg * C::kCols;
     const int KB = args.KB;
+    float* scr = reinterpret_cast<float*>(smem + C::kOffScr) + (warp - 4) * C::kCols;
     int tb = 0;
     uint32_t tphase = 0;
     bool ok = true;
@@ -356,6 +364,12 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
             break;
           }
           tc_fence_after();
+          if constexpr (kSwap) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+              if (32 * c + lane < C::kCols) scr[32 * c + lane] = ring_w[d] * ring_a[d][c];
+            __syncwarp();
+          }
           const uint32_t taddr =
               tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
 #pragma unroll
@@ -373,20 +387,30 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
                 for (int i = 0; i < 16; ++i) acc[c + 16 + i] = fmaf(sc, v1[i], acc[c + 16 + i]);
               }
             } else {
-              const float scv = ring_w[d] * ring_a[d][c / 32];
+              // column scales of this K-block, broadcast from the warp's slot
+              const float4* s4 = reinterpret_cast<const float4*>(scr + c);
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[c + i] = fmaf(__shfl_sync(0xffffffffu, scv, i), v0[i], acc[c + i]);
+              for (int i = 0; i < 4; ++i) {
+                const float4 q = s4[i];
+                acc[c + 4 * i + 0] = fmaf(q.x, v0[4 * i + 0], acc[c + 4 * i + 0]);
+                acc[c + 4 * i + 1] = fmaf(q.y, v0[4 * i + 1], acc[c + 4 * i + 1]);
+                acc[c + 4 * i + 2] = fmaf(q.z, v0[4 * i + 2], acc[c + 4 * i + 2]);
+                acc[c + 4 * i + 3] = fmaf(q.w, v0[4 * i + 3], acc[c + 4 * i + 3]);
+              }
               if (c + 16 < C::kCols) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  acc[c + 16 + i] =
-                      fmaf(__shfl_sync(0xffffffffu, scv, 16 + i), v1[i], acc[c + 16 + i]);
+                for (int i = 0; i < 4; ++i) {
+                  const float4 q = s4[4 + i];
+                  acc[c + 16 + 4 * i + 0] = fmaf(q.x, v1[4 * i + 0], acc[c + 16 + 4 * i + 0]);
+                  acc[c + 16 + 4 * i + 1] = fmaf(q.y, v1[4 * i + 1], acc[c + 16 + 4 * i + 1]);
+                  acc[c + 16 + 4 * i + 2] = fmaf(q.z, v1[4 * i + 2], acc[c + 16 + 4 * i + 2]);
+                  acc[c + 16 + 4 * i + 3] = fmaf(q.w, v1[4 * i + 3], acc[c + 16 + 4 * i + 3]);
+                }
               }
             }
           }
           tc_fence_before();
-          __syncwarp();
+          __syncwarp();   // also: every lane is done reading this K-block's scales
           if (lane == 0) mbar_arrive(&tempty[tb]);
           if (++tb == C::kBufs) {
             tb = 0;
@@ -440,9 +464,11 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
 
   if (args.splits > 1) {
     // ---------------------------------------- split-K reduction in the cluster --
-    // Each CTA publishes its fp32 partial tile [BN][128] (column-major in the
-    // MMA's row index) in its own (drained) stage memory; rank r then sums
-    // columns [r*BN/S, (r+1)*BN/S) over ranks 0..S-1 in order and writes Y.
+    // Each CTA publishes its fp32 partial tile [BN][128] (token-major, MMA row
+    // index contiguous) in its own drained stage memory; rank r then sums, over
+    // ranks 0..S-1 in that order, weight rows [4*(32r/S), 4*(32(r+1)/S)) of
+    // every valid token and writes those Y elements. (Only the swapped, decode
+    // order is ever split.)
     float* red = reinterpret_cast<float*>(smem);
     if (warp >= 4) {
       const int wg = (warp - 4) >> 2;
@@ -454,35 +480,38 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     cluster_sync();
     int last_rt, last_ct;  // split-K CTAs own exactly one tile: blockIdx.y
     tile_coords(blockIdx.y, args.row_tiles, args.col_tiles, last_rt, last_ct);
-    if (!*abort_flag) {
+    if (kSwap && !*abort_flag) {
       const int S = args.splits;
       const int rank = static_cast<int>(cluster_ctarank());
-      const int j_lo = rank * BN / S, j_hi = (rank + 1) * BN / S;
-      const int total4 = (j_hi - j_lo) * 32;
+      const int r_lo = 4 * (32 * rank / S), r_hi = 4 * (32 * (rank + 1) / S);
+      const int nr4 = (r_hi - r_lo) / 4;
+      const int tok_left = args.M - last_ct * BN;
+      const int n_tok = tok_left < BN ? tok_left : BN;
+      const int total4 = n_tok * nr4;
       for (int idx = threadIdx.x; idx < total4; idx += C::kThreads) {
-        const int j = j_lo + idx / 32;
-        const int r4 = (idx % 32) * 4;
+        const int j = idx / nr4;
+        const int r4 = r_lo + (idx - j * nr4) * 4;
         const uint32_t local = smem_u32(red + j * 128 + r4);
-        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < S; ++q) {
-          const float4 v = ld_cluster_f32x4(map_cluster(local, static_cast<uint32_t>(q)));
-          s.x += v.x;
-          s.y += v.y;
-          s.z += v.z;
-          s.w += v.w;
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) v[q] = ld_cluster_f32x4(map_cluster(local, static_cast<uint32_t>(q)));
+        float4 acc4 = v[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          if (q < S) {
+            acc4.x += v[q].x;
+            acc4.y += v[q].y;
+            acc4.z += v[q].z;
+            acc4.w += v[q].w;
+          }
         }
-        int out_row, out_col;  // Y coordinates of element (j, r4)
-        if constexpr (kSwap) {
-          out_row = last_ct * BN + j;
-          out_col = last_rt * 128 + r4;
-        } else {
-          out_row = last_rt * 128 + r4;  // (prefill split-K is not used)
-          out_col = last_ct * BN + j;
-        }
-        if (kSwap && out_row < args.M && out_col < args.N) {
+        const int out_row = last_ct * BN + j;       // token
+        const int out_col = last_rt * 128 + r4;     // weight row
+        if (out_col < args.N) {
           uint2 pk;
-          pk.x = pack_bf16x2(s.x, s.y);
-          pk.y = pack_bf16x2(s.z, s.w);
+          pk.x = pack_bf16x2(acc4.x, acc4.y);
+          pk.y = pack_bf16x2(acc4.z, acc4.w);
           *reinterpret_cast<uint2*>(args.y + static_cast<int64_t>(out_row) * args.N + out_col) =
               pk;
         }
@@ -501,9 +530,38 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
 
 // ------------------------------------------------------------------ host side --
 
+// How many clusters of `S` CTAs of `kern` can be resident at once (cached per
+// kernel, device and S).
+template <class Kern>
+int max_active_clusters(Kern kern, int threads, int smem, int S, int dev) {
+  static int cache[64][9];
+  static std::once_flag flags[64][9];
+  std::call_once(flags[dev][S], [&] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(S);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[dev][S] = n;
+  });
+  return cache[dev][S];
+}
+
 template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
                const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
+  // (grid_y, splits) as chosen by the shape heuristic; adjusted below.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   static std::once_flag flags[64];
@@ -516,22 +574,40 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
   });
   if (attr_err != cudaSuccess) return FP8BS_ERR_CUDA;
 
+  // A split launch needs every cluster resident at once (a cluster of S CTAs
+  // needs S free SMs of one GPC); shrink S until the clusters fit in one wave.
+  GemmArgs args = a;
+  while (splits > 1) {
+    const int fit = max_active_clusters(kern, C::kThreads, C::kSmemBytes, splits, dev);
+    if (fit >= grid_y) break;
+    --splits;
+    while (splits > 1 && args.KB / kKS < splits) --splits;
+  }
+  if (splits == 1 && args.splits > 1) {
+    DeviceInfo info;
+    if (current_device_info(&info) != FP8BS_OK) return FP8BS_ERR_CUDA;
+    grid_y = grid_y < info.sm_count ? grid_y : info.sm_count;   // persistent
+  }
+  args.splits = splits;
+
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(grid_y), 1);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attrs[1];
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
   if (splits > 1) {
-    attrs[0].id = cudaLaunchAttributeClusterDimension;
-    attrs[0].val.clusterDim.x = static_cast<unsigned>(splits);
-    attrs[0].val.clusterDim.y = 1;
-    attrs[0].val.clusterDim.z = 1;
-    cfg.attrs = attrs;
-    cfg.numAttrs = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = static_cast<unsigned>(splits);
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, te, a) != cudaSuccess) return FP8BS_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, te, args) != cudaSuccess) return FP8BS_ERR_CUDA;
   return FP8BS_OK;
 }
 

@@ -117,6 +117,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
     tma_prefetch_desc(&tmap_x);
   }
   __syncthreads();
+  // No global memory was touched so far; the input may come from the
+  // previous kernel of the stream.
+  grid_dependency_wait();
+  grid_launch_dependents();
   int issued = 0;
   if (t == 0) {
     for (int s = 0; s < kQStages; ++s) {
@@ -238,8 +242,17 @@ cudaError_t launch_stream(const void* x, int64_t rows, int64_t K, QArgs a, cudaS
   });
   if (attr != cudaSuccess) return attr;
   const int64_t ctas = a.num_tiles < 2LL * dev.sm_count ? a.num_tiles : 2LL * dev.sm_count;
-  kern<<<static_cast<unsigned>(ctas), kQThreads, kQSmemBytes, stream>>>(map, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = kQSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
 }  // namespace

@@ -189,7 +189,15 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   // Registers of the epilogue threads that outlive the role loop (split-K).
   float acc[C::kCols];
 
-  if (warp == 0) {
+  // Prefill: 384 threads launched at 168 registers (64512); the producer / MMA
+  // warpgroup drops to 40 and the two promotion warpgroups rise to 232
+  // (128 x 40 + 256 x 232 = 64512).
+  constexpr bool kRegSplit = !kSwap && kEpiWG == 2;
+  static_assert(!kRegSplit || C::kThreads == 384, "register split assumes 3 warpgroups");
+
+  if (warp < 4) {
+   if constexpr (kRegSplit) setmaxnreg_dec<40>();
+   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer --
       int stage = 0;
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
         mbar_wait(&full[s], ph, kDefaultWaitCycles);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     if (lane == 0) {
       // -------------------------------------------------------- MMA issuer --
       int stage = 0;
@@ -300,7 +308,9 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, kDefaultWaitCycles);
     }
-  } else if (warp >= 4) {
+   }
+  } else {
+    if constexpr (kRegSplit) setmaxnreg_inc<232>();
     // ------------------------------------------------- promotion / epilogue --
     const int wg = (warp - 4) >> 2;     // epilogue warpgroup
     const int quarter = warp & 3;       // TMEM lanes [32 quarter, 32 quarter + 32)
@@ -372,6 +382,20 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           }
           const uint32_t taddr =
               tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
+          if constexpr (!kSwap && C::kCols % 64 == 0) {
+            // prefill: 64 columns per TMEM round trip (two x32 loads, one wait)
+            const float sc = ring_a[d][0] * ring_w[d];
+#pragma unroll
+            for (int c = 0; c < C::kCols; c += 64) {
+              float v[64];
+              tmem_ld32(taddr + c, v);
+              tmem_ld32(taddr + c + 32, v + 32);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 64; i += 2)
+                fma2(acc[c + i], acc[c + i + 1], v[i], v[i + 1], sc, sc);
+            }
+          } else
 #pragma unroll
           for (int c = 0; c < C::kCols; c += 32) {
             float v0[16], v1[16];
@@ -392,19 +416,17 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const float4 q = s4[i];
-                acc[c + 4 * i + 0] = fmaf(q.x, v0[4 * i + 0], acc[c + 4 * i + 0]);
-                acc[c + 4 * i + 1] = fmaf(q.y, v0[4 * i + 1], acc[c + 4 * i + 1]);
-                acc[c + 4 * i + 2] = fmaf(q.z, v0[4 * i + 2], acc[c + 4 * i + 2]);
-                acc[c + 4 * i + 3] = fmaf(q.w, v0[4 * i + 3], acc[c + 4 * i + 3]);
+                fma2(acc[c + 4 * i], acc[c + 4 * i + 1], v0[4 * i], v0[4 * i + 1], q.x, q.y);
+                fma2(acc[c + 4 * i + 2], acc[c + 4 * i + 3], v0[4 * i + 2], v0[4 * i + 3], q.z,
+                     q.w);
               }
               if (c + 16 < C::kCols) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   const float4 q = s4[4 + i];
-                  acc[c + 16 + 4 * i + 0] = fmaf(q.x, v1[4 * i + 0], acc[c + 16 + 4 * i + 0]);
-                  acc[c + 16 + 4 * i + 1] = fmaf(q.y, v1[4 * i + 1], acc[c + 16 + 4 * i + 1]);
-                  acc[c + 16 + 4 * i + 2] = fmaf(q.z, v1[4 * i + 2], acc[c + 16 + 4 * i + 2]);
-                  acc[c + 16 + 4 * i + 3] = fmaf(q.w, v1[4 * i + 3], acc[c + 16 + 4 * i + 3]);
+                  float* a = acc + c + 16 + 4 * i;
+                  fma2(a[0], a[1], v1[4 * i], v1[4 * i + 1], q.x, q.y);
+                  fma2(a[2], a[3], v1[4 * i + 2], v1[4 * i + 3], q.z, q.w);
                 }
               }
             }
@@ -462,7 +484,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   tc_fence_before();
   __syncthreads();
 
-  if (args.splits > 1) {
+  if (kSwap && args.splits > 1) {
     // ---------------------------------------- split-K reduction in the cluster --
     // Each CTA publishes its fp32 partial tile [BN][128] (token-major, MMA row
     // index contiguous) in its own drained stage memory; rank r then sums, over

@@ -23,12 +23,39 @@ namespace fp8bs {
 struct ScaleDivider {
   float s;
   float r;
-  bool fast;
+  bool fast;      // Markstein allowed (per element checks still apply)
+  bool fast_all;  // branch-free codes allowed for every element (see codes2)
 
   __device__ __forceinline__ explicit ScaleDivider(float scale) : s(scale) {
     r = __frcp_rn(scale);
     // s normal (>= 2^-126) keeps r finite and normal for every bf16 amax.
     fast = scale >= 1.17549435e-38f && scale <= 1.0e37f;
+    fast_all = scale >= 8.27180613e-25f && scale <= 1.0e37f;  // s >= 2^-80
+  }
+
+  // Markstein's quotient without the range checks.
+  __device__ __forceinline__ float quotient_unchecked(float x) const {
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, s, x);
+    return __fmaf_rn(e, r, q0);
+  }
+
+  // E4M3 codes of two bf16 values packed as (lo, hi) halves of w, for s > 0.
+  // With s >= 2^-80 every element goes through quotient_unchecked on its
+  // magnitude and takes its sign bit from the input: the quotient is exact
+  // where it can be nonzero in E4M3 (|x| >= 2^-100 and |x / s| >= 2^-100),
+  // and everywhere else it is below 2^-20, far under the smallest E4M3
+  // subnormal, so the code is the signed zero either way. Smaller scales take
+  // the checked path.
+  __device__ __forceinline__ uint32_t codes2(uint32_t w) const {
+    const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
+    if (fast_all) {
+      const float q0 = quotient_unchecked(fabsf(x0)), q1 = quotient_unchecked(fabsf(x1));
+      const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+      return c | ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+    }
+    return __nv_cvt_float2_to_fp8x2(make_float2((*this)(x0), (*this)(x1)), __NV_SATFINITE,
+                                    __NV_E4M3);
   }
 
   __device__ __forceinline__ float operator()(float x) const {
@@ -73,7 +100,7 @@ __device__ __forceinline__ uint2 encode8(const uint4 v, const ScaleDivider& d) {
     return make_uint2(out[0], out[1]);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) out[i >> 1] |= e4m3x2(d, bf16_lo(w[i]), bf16_hi(w[i])) << ((i & 1) * 16);
+  for (int i = 0; i < 4; ++i) out[i >> 1] |= d.codes2(w[i]) << ((i & 1) * 16);
   return make_uint2(out[0], out[1]);
 }
 

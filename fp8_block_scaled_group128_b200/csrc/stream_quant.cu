@@ -12,8 +12,8 @@
 // All three are HBM streaming kernels. CTAs are persistent (two per SM); thread
 // 0 keeps a 3-deep ring of 32 KB tiles in flight with TMA
 // (cp.async.bulk.tensor, no swizzle, out-of-range rows read as zero), and all
-// 256 threads work from shared memory. Thread t owns the 16-byte chunk t % 16
-// of rows t/16 + 16 i (i = 0..7): 16 threads cover one 256-byte row, so every
+// 512 threads work from shared memory. Thread t owns the 16-byte chunk t % 16
+// of rows t/16 + 32 i (i = 0..3): 16 threads cover one 256-byte row, so every
 // global store of a warp is contiguous. The element quotient x / s is the IEEE
 // fp32 quotient (ScaleDivider) and the conversion is the hardware
 // cvt.rn.satfinite.e4m3x2.f32.
@@ -30,8 +30,10 @@ enum class QMode { kAct, kWeight, kPrune };
 
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
-constexpr int kQThreads = 256;
-constexpr int kQSmemBytes = kQStages * kTileBytes + 1024 + 256;
+constexpr int kQThreads = 512;
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kRowsPerThread = 128 * 16 / kQThreads;   // 16 threads per 256-byte row
+constexpr int kQSmemBytes = kQStages * kTileBytes + 1024 + 512;
 
 struct QArgs {
   int64_t rows;            // M (activations) or N (weights)
@@ -83,8 +85,7 @@ __device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d,
     packed = ((a0 & 0x8000u) ? 0x80u : 0u) | ((a1 & 0x8000u) ? 0x8000u : 0u) |
              ((b0 & 0x8000u) ? 0x800000u : 0u) | ((b1 & 0x8000u) ? 0x80000000u : 0u);
   } else {
-    packed = e4m3x2(d, __uint_as_float(a0 << 16), __uint_as_float(a1 << 16)) |
-             (e4m3x2(d, __uint_as_float(b0 << 16), __uint_as_float(b1 << 16)) << 16);
+    packed = d.codes2(a0 | (a1 << 16)) | (d.codes2(b0 | (b1 << 16)) << 16);
   }
   // pruned weights: keep positions i0, i1 of each group, +0 elsewhere
   const uint64_t m0 = (0xFFFFull << (16 * (n0 & 3u))) | (0xFFFFull << (16 * (n0 >> 2)));
@@ -102,8 +103,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kTileBytes);
-  float* red = reinterpret_cast<float*>(full + kQStages);   // [2][8] block-max partials
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 16);
+  float* red = reinterpret_cast<float*>(full + kQStages);   // [2][kQWarps] block-max partials
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kQWarps);
 
   const int t = threadIdx.x;
   const int chunk = t & 15;
@@ -142,19 +143,20 @@ __global__ void __launch_bounds__(kQThreads, 2)
       record_device_error(a.err, FP8BS_ERR_DEVICE_TIMEOUT);
       *abort_flag = 1;
     }
-    uint4 v[8];
+    uint4 v[kRowsPerThread];
     const uint8_t* buf = smem + s * kTileBytes;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      v[i] = *reinterpret_cast<const uint4*>(buf + (i * 16 + (t >> 4)) * 256 + chunk * 16);
+    for (int i = 0; i < kRowsPerThread; ++i)
+      v[i] = *reinterpret_cast<const uint4*>(buf + (i * (kQThreads / 16) + (t >> 4)) * 256 +
+                                             chunk * 16);
 
     float m = 0.0f;
     if constexpr (kMode != QMode::kAct) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, amax8(v[i]));
+      for (int i = 0; i < kRowsPerThread; ++i) m = fmaxf(m, amax8(v[i]));
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if ((t & 31) == 0) red[(it & 1) * 8 + (t >> 5)] = m;
+      if ((t & 31) == 0) red[(it & 1) * kQWarps + (t >> 5)] = m;
     }
     // Every thread has read stage s (and published its block-max partial);
     // the proxy fence orders those reads before the TMA that refills stage s.
@@ -174,11 +176,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
     if constexpr (kMode == QMode::kAct) {
       // one 1x128 group per row: 16 threads hold a row
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kRowsPerThread; ++i) {
         float rm = amax8(v[i]);
 #pragma unroll
         for (int off = 8; off >= 1; off >>= 1) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, off));
-        const int64_t r = rb * 128 + i * 16 + (t >> 4);
+        const int64_t r = rb * 128 + i * (kQThreads / 16) + (t >> 4);
         const float sc = __fdiv_rn(rm, 448.0f);
         if (r < a.rows) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], ScaleDivider(sc));
@@ -186,15 +188,15 @@ __global__ void __launch_bounds__(kQThreads, 2)
         }
       }
     } else {
-      m = red[(it & 1) * 8];
+      m = red[(it & 1) * kQWarps];
 #pragma unroll
-      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[(it & 1) * 8 + w]);
+      for (int w = 1; w < kQWarps; ++w) m = fmaxf(m, red[(it & 1) * kQWarps + w]);
       const float sc = __fdiv_rn(m, 448.0f);
       if (t == 0) a.scale[rb * KB + kb] = sc;
       const ScaleDivider d(sc);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t r = rb * 128 + i * 16 + (t >> 4);
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int64_t r = rb * 128 + i * (kQThreads / 16) + (t >> 4);
         if (r >= a.rows) continue;
         if constexpr (kMode == QMode::kWeight) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], d);

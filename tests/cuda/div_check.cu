@@ -1,7 +1,8 @@
 // Exhaustive check of the library's scale division (ScaleDivider) against
 // CUDA's IEEE division __fdiv_rn, over the whole domain the quantizers use:
 // s = fl32(amax / 448) for every positive finite bf16 amax, and every finite
-// bf16 x with |x| <= amax (both signs). Also checks the E4M3 codes.
+// bf16 x with |x| <= amax (both signs). Also checks the E4M3 codes, both of
+// the checked quotient and of the quantizers' branch-free pair path.
 #include <cstdint>
 
 #include "../../fp8_block_scaled_group128_b200/csrc/e4m3_codec.cuh"
@@ -36,7 +37,9 @@ __global__ void div_check_kernel(Result* res) {
     }
     const uint32_t c = __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
     const uint32_t c_ref = __nv_cvt_float_to_fp8(q_ref, __NV_SATFINITE, __NV_E4M3);
-    bad_c += c != c_ref;
+    // the quantizers' pair path (x in the low half, +0 in the high half)
+    const uint32_t c2 = d.codes2(xb) & 0xFFu;
+    bad_c += (c != c_ref) + (c2 != c_ref);
   }
   atomicAdd(&res->checked, n);
   if (bad_q) atomicAdd(&res->quotient_mismatch, bad_q);

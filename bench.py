@@ -7,8 +7,8 @@ down (4096, 14336); tokens M in {1, 8, 32, 128}):
 
   1. weight quantization of the four bf16 weights (128x128 blocks)
   2. 2:4 prune + compress of the four weights
-  3. for each M, for each linear: activation quantization (1x128 groups),
-     dense block-scaled GEMM, 2:4 sparse block-scaled GEMM
+  3. for each M: the four activation quantizations (1x128 groups), the four
+     dense block-scaled GEMMs, the four 2:4 sparse block-scaled GEMMs
 
 The metric is HBM throughput of the step (algorithmic bytes of every launch /
 device time), with the dominant kernel's roofline fraction against the
@@ -17,7 +17,12 @@ per-step working set (~2.7 GB) is far larger than L2 and every weight is
 re-read only after more than L2's worth of other traffic. The step is
 captured once as a CUDA graph and replayed, so host launch cost stays out of
 the device timing; the last steps of the timed region use copies of the graph
-with an event between launches, for the per-kernel split.
+with an event wherever the launch kind changes, for the per-kernel split.
+
+The same JSON line also carries a "prefill" section: the dense GEMM on the
+prefill-shaped linears (M in {2048, 8192}, the four Llama-3-8B linears and
+the LM head) and the 2:4 GEMM at M = 4096, in TFLOP/s against the dense FP8
+tensor peak.
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -74,12 +79,15 @@ def kernel_bytes(kind, M, N, K):
 
 
 def step_launches():
-    """(kind, M, N, K) of every launch of one step, in issue order."""
+    """(kind, M, N, K) of every launch of one step, in issue order: the weight
+    rows, then per token count M the four activation quantizations, the four
+    dense GEMMs and the four 2:4 GEMMs (same-kind launches back to back, so
+    the live per-kernel split needs an event only where the kind changes)."""
     out = [("quant_weight", 0, N, K) for N, K in LINEARS]
     out += [("prune24", 0, N, K) for N, K in LINEARS]
     for M in TOKENS:
-        for N, K in LINEARS:
-            out += [("quant_act", M, 0, K), ("dense_gemm", M, N, K), ("sparse_gemm", M, N, K)]
+        for kind in ("quant_act", "dense_gemm", "sparse_gemm"):
+            out += [(kind, M, N, K) for N, K in LINEARS]
     return [l for l in out if l[0] in ROWS]
 
 
@@ -99,9 +107,11 @@ class Step:
         self.x = {}
         for N, K in LINEARS:
             self.w[(N, K)] = synth.weights("llama", N, K, seed=seed).to(device)
+        # one activation per (M, linear), as the inputs of a layer's four
+        # linears are four different tensors
         for M in TOKENS:
-            for K in sorted({K for _, K in LINEARS}):
-                self.x[(M, K)] = synth.activations("llama", M, K, seed=seed).to(device)
+            for i, (N, K) in enumerate(LINEARS):
+                self.x[(M, N, K)] = synth.activations("llama", M, K, seed=seed + 101 * i).to(device)
         e = lambda *s, dt: torch.empty(*s, dtype=dt, device=device)  # noqa: E731
         self.qw, self.sw, self.vals, self.meta, self.sws = {}, {}, {}, {}, {}
         for N, K in LINEARS:
@@ -114,8 +124,8 @@ class Step:
         self.qa, self.sa, self.y, self.ys = {}, {}, {}, {}
         for M in TOKENS:
             for N, K in LINEARS:
-                self.qa[(M, K)] = e(M, K, dt=torch.uint8)
-                self.sa[(M, K)] = e(M, K // 128, dt=torch.float32)
+                self.qa[(M, N, K)] = e(M, K, dt=torch.uint8)
+                self.sa[(M, N, K)] = e(M, K // 128, dt=torch.float32)
                 self.y[(M, N, K)] = e(M, N, dt=torch.bfloat16)
                 self.ys[(M, N, K)] = e(M, N, dt=torch.bfloat16)
 
@@ -132,14 +142,16 @@ class Step:
                 sw=self.sws[(N, K)])))
         for M in TOKENS:
             for N, K in LINEARS:
-                out.append(("quant_act", lambda M=M, K=K: fb.fp8_quant_act_group128(
-                    self.x[(M, K)], qa=self.qa[(M, K)], sa=self.sa[(M, K)])))
+                out.append(("quant_act", lambda M=M, N=N, K=K: fb.fp8_quant_act_group128(
+                    self.x[(M, N, K)], qa=self.qa[(M, N, K)], sa=self.sa[(M, N, K)])))
+            for N, K in LINEARS:
                 out.append(("dense_gemm", lambda M=M, N=N, K=K: fb.fp8_block_gemm(
-                    self.qa[(M, K)], self.sa[(M, K)], self.qw[(N, K)], self.sw[(N, K)],
+                    self.qa[(M, N, K)], self.sa[(M, N, K)], self.qw[(N, K)], self.sw[(N, K)],
                     y=self.y[(M, N, K)])))
+            for N, K in LINEARS:
                 out.append(("sparse_gemm", lambda M=M, N=N, K=K: fb.fp8_sparse24_gemm(
-                    self.qa[(M, K)], self.sa[(M, K)], self.vals[(N, K)], self.meta[(N, K)],
-                    self.sws[(N, K)], y=self.ys[(M, N, K)])))
+                    self.qa[(M, N, K)], self.sa[(M, N, K)], self.vals[(N, K)],
+                    self.meta[(N, K)], self.sws[(N, K)], y=self.ys[(M, N, K)])))
         return [(k, f) for k, f in out if k in ROWS]
 
     def run(self):
@@ -285,6 +297,84 @@ def barrier(world):
         dist.barrier()
 
 
+# ------------------------------------------------------------- prefill --
+
+def fp8_tensor_peak():
+    """Dense FP8 tensor peak (TFLOP/s): the measured cuBLAS bf16 burst figure
+    times 2, the nominal fp8 : bf16 dense ratio of B200 (4.5 : 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2"
+    except (OSError, KeyError, ValueError):
+        return 2.0 * 1590.0, "fallback bf16 1.59 PF/s x 2"
+
+
+def run_prefill(dev, stream, world, reps=10):
+    """Prefill-shaped GEMMs timed on their own: the dense GEMM at M in {2048,
+    8192} on the four Llama-3-8B linears and the LM head, and the 2:4 GEMM at
+    M = 4096 on its two shapes. Each shape's launches are replayed from a CUDA
+    graph of `reps` back-to-back launches (one warm-up replay, three timed),
+    CUDA events on the launching stream. Inputs: the seeded synthetic llama
+    tensors, quantized / compressed on the device before timing."""
+    from fp8_block_scaled_group128_b200 import binding as fb
+    from fp8_block_scaled_group128_b200 import synth
+    peak, peak_src = fp8_tensor_peak()
+    shapes = [("dense", M, N, K) for M in synth.PREFILL_M
+              for N, K in synth.LLAMA3_8B_LINEARS + (synth.LLAMA3_8B_LM_HEAD,)]
+    shapes += [("sparse", 4096, N, K) for N, K in synth.SPARSE_LINEARS]
+    rows, tot_flop, tot_ms = [], 0.0, 0.0
+    wcache = {}
+    for kind, M, N, K in shapes:
+        with torch.cuda.stream(stream):
+            key = (kind, N, K)
+            if key not in wcache:
+                wcache.clear()
+                w = synth.weights("llama", N, K, seed=7).to(dev)
+                wcache[key] = (fb.fp8_quant_weight_block128(w) if kind == "dense"
+                               else fb.prune24_compress(w)[:3])
+                del w
+            x = synth.activations("llama", M, K, seed=7).to(dev)
+            qa, sa = fb.fp8_quant_act_group128(x)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            wq = wcache[key]
+            fn = ((lambda: fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y)) if kind == "dense" else
+                  (lambda: fb.fp8_sparse24_gemm(qa, sa, wq[0], wq[1], wq[2], y=y)))
+            fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record()
+            for _ in range(3):
+                g.replay()
+            e1.record()
+        stream.synchronize()
+        assert fb.get_device_error(stream) == 0
+        ms = max_over_ranks(e0.elapsed_time(e1) / (3 * reps), world)
+        # algorithmic FLOPs: 2MNK dense; MNK (the kept half) for 2:4
+        flop = (2.0 if kind == "dense" else 1.0) * M * N * K
+        tf = flop / (ms * 1e-3) / 1e12
+        rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
+                     "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4)})
+        if kind == "dense":
+            tot_flop += flop
+            tot_ms += ms
+        del g, x, qa, sa, y
+    wcache.clear()
+    torch.cuda.empty_cache()
+    agg = tot_flop / (tot_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
+            "dense_achieved": round(agg, 1), "dense_frac": round(agg / peak, 4),
+            "note": "dense: 2MNK FLOPs; 2:4: MNK FLOPs (nonzero work) against the dense peak",
+            "shapes": rows}
+
+
 # ------------------------------------------------------------ CPU side --
 
 def oracle_sample(budget_s=15.0):
@@ -348,25 +438,33 @@ def run_ours(args, rank, world, local):
 
     # The step is captured as one CUDA graph and replayed (host launch cost
     # stays out of the device timing). The last R steps of the timed region
-    # replay copies of the graph that also hold an event record node between
-    # consecutive launches (external events), each copy its own events: every
-    # launch's device time over those R steps is measured live inside the timed
-    # region. Event nodes cost a few microseconds each, so the other steps run
-    # the plain graph.
+    # replay copies of the graph that also hold an event record node wherever
+    # the launch kind changes (external events; each copy its own events):
+    # every kind's device time over those R steps is measured live inside the
+    # timed region, a run of same-kind launches as one span. Event nodes cost
+    # a few microseconds each, so the other steps run the plain graph.
     R = min(10, args.steps)
     launches_fns = step.launches()
+    # (kind, index of the first launch, index past the last) of each run
+    groups = []
+    for i, (kind, _) in enumerate(launches_fns):
+        if groups and groups[-1][0] == kind:
+            groups[-1][2] = i + 1
+        else:
+            groups.append([kind, i, i + 1])
 
     def capture(with_events):
         evs = [torch.cuda.Event(enable_timing=True, external=True)
-               for _ in range(len(launches_fns) + 1)] if with_events else None
+               for _ in range(len(groups) + 1)] if with_events else None
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             if evs:
                 evs[0].record()
-            for i, (_, fn) in enumerate(launches_fns):
-                fn()
+            for gi, (_, a, b) in enumerate(groups):
+                for _, fn in launches_fns[a:b]:
+                    fn()
                 if evs:
-                    evs[i + 1].record()
+                    evs[gi + 1].record()
         return g, evs
 
     plain, _ = capture(False)
@@ -396,8 +494,8 @@ def run_ours(args, rank, world, local):
     total_ms = t0.elapsed_time(t1)
     kernel_ms = {k: 0.0 for k in ROWS}
     for _, evs in evented:
-        for i, (kind, _) in enumerate(launches_fns):
-            kernel_ms[kind] += evs[i].elapsed_time(evs[i + 1]) / R
+        for gi, (kind, _, _) in enumerate(groups):
+            kernel_ms[kind] += evs[gi].elapsed_time(evs[gi + 1]) / R
     assert fb.get_device_error(stream) == 0
     ms_step = max_over_ranks(total_ms / args.steps, world)
 
@@ -470,6 +568,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": WORKLOAD, "rows": list(ROWS), "linears_NK": [list(l) for l in LINEARS],
                    "tokens_M": list(TOKENS), "global_batch": sum(TOKENS) * world,
                    "step_bytes": sb, "launches_per_step": per_step_launches,
+                   "event_nodes_per_evented_step": len(groups) + 1,
                    "parallelism": f"replicas x{world} (token data parallel, no collective)",
                    "l2": "working set per step ~2.7 GB >> 126 MB L2; every weight is re-read "
                          "only after >126 MB of other traffic; CUDA-graph replay"},
@@ -479,6 +578,8 @@ def run_ours(args, rank, world, local):
         "gpu_launches": per_step_launches * args.steps,
         "clocks": clocks.summary(),
     }
+    if not args.no_prefill:
+        result["prefill"] = run_prefill(dev, stream, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, el, desc, cores = oracle_sample(args.cpu_budget)
         result["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores,
@@ -525,6 +626,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill-shaped GEMM section of the JSON line")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -1,0 +1,99 @@
+"""Run one step of the path on one shape, a few times, for a profiler.
+
+    python -m fp8_block_scaled_group128_b200.profile_case KIND M N K ITERS
+
+KIND is one of quant_act, quant_weight, prune24, dense_gemm, sparse_gemm.
+The inputs are the seeded synthetic llama tensors of that shape, prepared on
+the device by the library's own kernels before the ITERS launches of the
+kernel under test (select those with the profiler's kernel-name filter).
+Prints the mean device time of the ITERS launches (CUDA events).
+
+    python -m fp8_block_scaled_group128_b200.profile_case decode_step ITERS
+
+runs ITERS passes of the decode step's launches in issue order (the weight
+rows of the four Llama-3-8B linears, then per M in {1, 8, 32, 128} the four
+activation quantizations, dense GEMMs and 2:4 GEMMs), with about 0.9 GB on
+the device.
+"""
+
+import sys
+
+import torch
+
+from . import binding as fb
+from . import synth
+
+
+def decode_step(iters):
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    lin = synth.LLAMA3_8B_LINEARS
+    w = {nk: synth.weights("llama", *nk, seed=0).to(dev) for nk in lin}
+    x = {(M, nk): synth.activations("llama", M, nk[1], seed=0).to(dev)
+         for M in synth.DECODE_M for nk in lin}
+    for _ in range(iters):
+        q = {nk: fb.fp8_quant_weight_block128(w[nk]) for nk in lin}
+        s = {nk: fb.prune24_compress(w[nk])[:3] for nk in lin}
+        for M in synth.DECODE_M:
+            a = {nk: fb.fp8_quant_act_group128(x[(M, nk)]) for nk in lin}
+            for nk in lin:
+                fb.fp8_block_gemm(*a[nk], *q[nk])
+            for nk in lin:
+                fb.fp8_sparse24_gemm(*a[nk], *s[nk])
+    torch.cuda.synchronize()
+    if fb.get_device_error() != 0:
+        raise SystemExit("device error")
+    print(f"decode_step: {iters} passes")
+
+
+def main(argv):
+    if argv[0] == "decode_step":
+        return decode_step(int(argv[1]))
+    kind, M, N, K, iters = argv[0], int(argv[1]), int(argv[2]), int(argv[3]), int(argv[4])
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if kind in ("quant_weight", "prune24", "dense_gemm", "sparse_gemm"):
+        w = synth.weights("llama", N, K, seed=0).to(dev)
+    if kind in ("quant_act", "dense_gemm", "sparse_gemm"):
+        x = synth.activations("llama", max(M, 1), K, seed=0).to(dev)
+
+    if kind == "quant_act":
+        qa = torch.empty(M, K, dtype=torch.uint8, device=dev)
+        sa = torch.empty(M, K // 128, dtype=torch.float32, device=dev)
+        fn = lambda: fb.fp8_quant_act_group128(x, qa=qa, sa=sa)  # noqa: E731
+    elif kind == "quant_weight":
+        qw = torch.empty(N, K, dtype=torch.uint8, device=dev)
+        sw = torch.empty(-(-N // 128), K // 128, dtype=torch.float32, device=dev)
+        fn = lambda: fb.fp8_quant_weight_block128(w, qw=qw, sw=sw)  # noqa: E731
+    elif kind == "prune24":
+        vals = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+        meta = torch.empty(N, K // 8, dtype=torch.uint8, device=dev)
+        sw = torch.empty(-(-N // 128), K // 128, dtype=torch.float32, device=dev)
+        fn = lambda: fb.prune24_compress(w, vals=vals, meta=meta, sw=sw)  # noqa: E731
+    elif kind in ("dense_gemm", "sparse_gemm"):
+        qa, sa = fb.fp8_quant_act_group128(x)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        if kind == "dense_gemm":
+            qw, sw = fb.fp8_quant_weight_block128(w)
+            fn = lambda: fb.fp8_block_gemm(qa, sa, qw, sw, y=y)  # noqa: E731
+        else:
+            vals, meta, sw, _ = fb.prune24_compress(w)
+            fn = lambda: fb.fp8_sparse24_gemm(qa, sa, vals, meta, sw, y=y)  # noqa: E731
+        del w
+    else:
+        raise SystemExit(f"unknown kind {kind!r}")
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if fb.get_device_error() != 0:
+        raise SystemExit("device error")
+    print(f"{kind} M={M} N={N} K={K}: {e0.elapsed_time(e1) / iters * 1e3:.2f} us/launch "
+          f"over {iters} launches")
+
+
+if __name__ == "__main__":
+    main(sys.argv[1:])

@@ -11,26 +11,72 @@
 // underflows. The reciprocal is computed once per scale; elements that are
 // zero or tiny (|x| < 2^-100), whose quotient is tiny (|x r| < 2^-100, where
 // the quotient could be subnormal) or whose scale is subnormal take the IEEE
-// division __fdiv_rn instead. tests/test_gpu_division.py checks the result
-// bit for bit against __fdiv_rn for every bf16 amax and every bf16 x with
-// |x| <= amax.
+// division __fdiv_rn instead. The scale itself, amax / 448, is formed the
+// same way with the divisor 448. tests/cuda/div_check.cu checks all of it bit
+// for bit against __fdiv_rn: the scale for every bf16 amax, and the quotient
+// and codes (scalar and packed paths) for every bf16 amax and every bf16 x
+// with |x| <= amax.
 #pragma once
 
 #include "common.cuh"
 
 namespace fp8bs {
 
+// Byte permute (PTX prmt.b32, default mode): selector nibble bits 0-2 pick one
+// of the 8 bytes {b, a}; bit 3 set replicates that byte's sign bit instead.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Per 16-bit half: a bf16 whose magnitude is max(|a|, |b|). The sign bits of
+// the result are meaningless (mask them before use).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Largest magnitude (as fp32) of the two halves of a bf16x2 absmax word.
+__device__ __forceinline__ float absmax_to_float(uint32_t m2) {
+  const uint32_t m = m2 & 0x7FFF7FFFu;
+  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+  return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+
+// s = fl32(amax / 448), correctly rounded, for a finite amax >= 0.
+__device__ __forceinline__ float scale_of_amax(float amax) {
+  if (amax >= 7.88860905e-31f) {  // 2^-100: quotient and residual stay normal
+    const float r = __frcp_rn(448.0f);
+    const float q0 = __fmul_rn(amax, r);
+    const float e = __fmaf_rn(-q0, 448.0f, amax);
+    return __fmaf_rn(e, r, q0);
+  }
+  return __fdiv_rn(amax, 448.0f);
+}
+
 struct ScaleDivider {
   float s;
   float r;
-  bool fast;      // Markstein allowed (per element checks still apply)
-  bool fast_all;  // branch-free codes allowed for every element (see codes2)
+  bool fast;       // Markstein allowed (per element checks still apply)
+  bool fast_all;   // branch-free codes allowed for every element (see codes2)
+  uint64_t r2;     // (r, r) packed for fp32x2 arithmetic
+  uint64_t ns2;    // (-s, -s)
 
   __device__ __forceinline__ explicit ScaleDivider(float scale) : s(scale) {
     r = __frcp_rn(scale);
     // s normal (>= 2^-126) keeps r finite and normal for every bf16 amax.
     fast = scale >= 1.17549435e-38f && scale <= 1.0e37f;
     fast_all = scale >= 8.27180613e-25f && scale <= 1.0e37f;  // s >= 2^-80
+    r2 = pack_f32x2(r, r);
+    ns2 = pack_f32x2(-scale, -scale);
   }
 
   // Markstein's quotient without the range checks.
@@ -40,22 +86,53 @@ struct ScaleDivider {
     return __fmaf_rn(e, r, q0);
   }
 
-  // E4M3 codes of two bf16 values packed as (lo, hi) halves of w, for s > 0.
-  // With s >= 2^-80 every element goes through quotient_unchecked on its
-  // magnitude and takes its sign bit from the input: the quotient is exact
-  // where it can be nonzero in E4M3 (|x| >= 2^-100 and |x / s| >= 2^-100),
-  // and everywhere else it is below 2^-20, far under the smallest E4M3
-  // subnormal, so the code is the signed zero either way. Smaller scales take
-  // the checked path.
+  // The same on two values at once (fp32x2 instructions; each lane rounds
+  // exactly like the scalar form, since q0 * (-s) + x == -q0 * s + x).
+  __device__ __forceinline__ void quotient2_unchecked(float x0, float x1, float& q0,
+                                                      float& q1) const {
+    asm("{\n\t.reg .b64 x, q, e;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mul.rn.f32x2 q, x, %4;\n\t"
+        "fma.rn.f32x2 e, q, %5, x;\n\t"
+        "fma.rn.f32x2 q, e, %4, q;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(q0), "=f"(q1)
+        : "f"(x0), "f"(x1), "l"(r2), "l"(ns2));
+  }
+
+  // E4M3 codes of the magnitudes of two bf16 values packed as (lo, hi) halves
+  // of w (lo -> byte 0), through the unchecked quotient (fast_all only).
+  __device__ __forceinline__ uint32_t mag_codes2(uint32_t w) const {
+    const uint32_t a = w & 0x7FFF7FFFu;
+    float q0, q1;
+    quotient2_unchecked(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u), q0, q1);
+    return __nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+  }
+
+  // E4M3 codes of two bf16 values packed as (lo, hi) halves of w, for s > 0
+  // (x0 = lo -> byte 0). With s >= 2^-80 both elements go through the
+  // unchecked quotient of their magnitudes and take their sign bit from the
+  // input: the quotient is exact where it can be nonzero in E4M3 (|x| >=
+  // 2^-100 and |x / s| >= 2^-100), and everywhere else it is below 2^-20, far
+  // under the smallest E4M3 subnormal, so the code is the signed zero either
+  // way. Smaller scales take the checked path.
   __device__ __forceinline__ uint32_t codes2(uint32_t w) const {
-    const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
     if (fast_all) {
-      const float q0 = quotient_unchecked(fabsf(x0)), q1 = quotient_unchecked(fabsf(x1));
-      const uint32_t c = __nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
-      return c | ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
+      // byte 0 <- sign of the low bf16 (bit 15), byte 1 <- sign of the high one
+      return mag_codes2(w) | (prmt(w, 0u, 0x44B9u) & 0x8080u);
     }
+    const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
     return __nv_cvt_float2_to_fp8x2(make_float2((*this)(x0), (*this)(x1)), __NV_SATFINITE,
                                     __NV_E4M3);
+  }
+
+  // Four codes: the two of w0 in bytes 0-1, the two of w1 in bytes 2-3.
+  __device__ __forceinline__ uint32_t codes4(uint32_t w0, uint32_t w1) const {
+    if (fast_all) {
+      // the four input sign bits (bits 15, 31 of w0 and of w1), replicated
+      return prmt(mag_codes2(w0), mag_codes2(w1), 0x5410u) | (prmt(w0, w1, 0xFDB9u) & 0x80808080u);
+    }
+    return prmt(codes2(w0), codes2(w1), 0x5410u);
   }
 
   __device__ __forceinline__ float operator()(float x) const {
@@ -71,49 +148,21 @@ struct ScaleDivider {
   }
 };
 
-// Two codes (x0 in the low byte) for a nonzero scale.
-__device__ __forceinline__ uint32_t e4m3x2(const ScaleDivider& d, float x0, float x1) {
-  return __nv_cvt_float2_to_fp8x2(make_float2(d(x0), d(x1)), __NV_SATFINITE, __NV_E4M3);
+// Codes of two bf16 pairs (as codes4) for a zero scale (an all-zero group or
+// block): each element's signed zero.
+__device__ __forceinline__ uint32_t zero_codes4(uint32_t w0, uint32_t w1) {
+  return prmt(w0, w1, 0xFDB9u) & 0x80808080u;
 }
-
-// One code; a zero scale (all-zero group or block) gives the element's signed zero.
-__device__ __forceinline__ uint32_t e4m3_code_bf16(const ScaleDivider& d, uint32_t bf16_bits) {
-  if (d.s == 0.0f) return (bf16_bits & 0x8000u) ? 0x80u : 0x00u;
-  const float x = __uint_as_float(bf16_bits << 16);
-  return static_cast<uint32_t>(__nv_cvt_float_to_fp8(d(x), __NV_SATFINITE, __NV_E4M3));
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Encode 8 bf16 values (a uint4) into 8 E4M3 bytes (a uint2).
 __device__ __forceinline__ uint2 encode8(const uint4 v, const ScaleDivider& d) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[2] = {0u, 0u};
-  if (d.s == 0.0f) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = (w[i] & 0x8000u) ? 0x80u : 0u;
-      const uint32_t hi = (w[i] & 0x80000000u) ? 0x80u : 0u;
-      out[i >> 1] |= (lo | (hi << 8)) << ((i & 1) * 16);
-    }
-    return make_uint2(out[0], out[1]);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) out[i >> 1] |= d.codes2(w[i]) << ((i & 1) * 16);
-  return make_uint2(out[0], out[1]);
+  if (d.s == 0.0f) return make_uint2(zero_codes4(v.x, v.y), zero_codes4(v.z, v.w));
+  return make_uint2(d.codes4(v.x, v.y), d.codes4(v.z, v.w));
 }
 
-// Largest |x| of 8 bf16 values.
-__device__ __forceinline__ float amax8(const uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, fabsf(bf16_lo(w[i])));
-    m = fmaxf(m, fabsf(bf16_hi(w[i])));
-  }
-  return m;
+// bf16x2 absmax word of 8 bf16 values (see absmax_to_float).
+__device__ __forceinline__ uint32_t absmax8(const uint4 v) {
+  return bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w));
 }
 
 }  // namespace fp8bs

@@ -26,7 +26,8 @@ namespace fp8bs {
 
 namespace {
 
-enum class QMode { kAct, kWeight, kPrune };
+// kPruneOut: 2:4 prune + compress that also writes the pruned bf16 weights.
+enum class QMode { kAct, kWeight, kPrune, kPruneOut };
 
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
@@ -48,52 +49,61 @@ struct QArgs {
   int* err;
 };
 
-// 2:4 selection of one group of 4 bf16 values held in a 64-bit word (value j
-// in bits 16j..16j+15). Each member gets the key (|w| bits << 2) | (3 - j):
-// a larger magnitude wins, and equal magnitudes go to the lower index. The two
-// largest keys (a 4-input max / second-max network) are the kept pair.
-// Returns i0 | i1 << 2 (i0 < i1) and the two kept bf16 patterns in position
-// order.
-__device__ __forceinline__ uint32_t select24(uint64_t g, uint32_t& k0, uint32_t& k1) {
-  uint32_t key[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    key[j] = ((static_cast<uint32_t>(g >> (16 * j)) & 0x7FFFu) << 2) | static_cast<uint32_t>(3 - j);
-  const uint32_t a = max(key[0], key[1]), b = min(key[0], key[1]);
-  const uint32_t c = max(key[2], key[3]), d = min(key[2], key[3]);
-  const uint32_t top1 = max(a, c);
-  const uint32_t top2 = max(min(a, c), max(b, d));
-  const uint32_t p1 = 3u - (top1 & 3u), p2 = 3u - (top2 & 3u);
-  const uint32_t i0 = min(p1, p2), i1 = max(p1, p2);
-  k0 = static_cast<uint32_t>(g >> (16 * i0)) & 0xFFFFu;
-  k1 = static_cast<uint32_t>(g >> (16 * i1)) & 0xFFFFu;
-  return i0 | (i1 << 2);
-}
-
-// 2:4 selection and encoding of the 8 weights (two groups) of one thread-row:
-// returns the 4 value bytes, sets the metadata byte and the pruned bf16 words.
-__device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d, uint32_t& nib2,
+// 2:4 selection, metadata and codes of the 8 weights (two groups of 4 along
+// K) in one 16-byte chunk: group 0 in v.x (elements 0, 1) and v.y (2, 3),
+// group 1 in v.z and v.w. Element j "beats" element i when |w_j| > |w_i|, or
+// |w_j| == |w_i| and j < i; an element is kept when at most one other beats
+// it, which keeps exactly two per group.
+//
+// Both groups are ranked at once in 16-bit lanes: E_j pairs element j of
+// group 0 (low half) with element j of group 1 (high half); for i < j,
+// (E_i | 0x8000 per lane) - |E_j| leaves bit 15 of each lane set exactly when
+// |w_i| >= |w_j| (15-bit magnitudes, no borrow between the lanes). Each kept
+// flag is then the majority of three such bits.
+//
+// Returns the 4 value bytes (kept codes of group 0 in position order, then
+// group 1); sets the metadata byte (group 0 nibble in bits 0-3, group 1 in
+// 4-7, nibble = i0 | i1 << 2) and, if kPruned, the pruned bf16 chunk.
+template <bool kPruned>
+__device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d, uint32_t& meta,
                                            uint4& pruned) {
-  const uint64_t g0 = (static_cast<uint64_t>(v.y) << 32) | v.x;
-  const uint64_t g1 = (static_cast<uint64_t>(v.w) << 32) | v.z;
-  uint32_t a0, a1, b0, b1;
-  const uint32_t n0 = select24(g0, a0, a1);
-  const uint32_t n1 = select24(g1, b0, b1);
-  nib2 = n0 | (n1 << 4);
-  uint32_t packed;
-  if (d.s == 0.0f) {
-    packed = ((a0 & 0x8000u) ? 0x80u : 0u) | ((a1 & 0x8000u) ? 0x8000u : 0u) |
-             ((b0 & 0x8000u) ? 0x800000u : 0u) | ((b1 & 0x8000u) ? 0x80000000u : 0u);
-  } else {
-    packed = d.codes2(a0 | (a1 << 16)) | (d.codes2(b0 | (b1 << 16)) << 16);
+  const uint32_t e0 = prmt(v.x, v.z, 0x5410u), e1 = prmt(v.x, v.z, 0x7632u);
+  const uint32_t e2 = prmt(v.y, v.w, 0x5410u), e3 = prmt(v.y, v.w, 0x7632u);
+  constexpr uint32_t kTop = 0x80008000u;
+  const uint32_t g0 = e0 | kTop, g1 = e1 | kTop, g2 = e2 | kTop, g3 = e3 | kTop;
+  // c_ij (bit 15 / 31): |w_i| >= |w_j|, i.e. i beats j (i < j); per lane
+  // (0x8000 + |w_i|) - (0x8000 + |w_j|) + 0x8000
+  const uint32_t c01 = g0 - g1 + kTop, c02 = g0 - g2 + kTop, c03 = g0 - g3 + kTop;
+  const uint32_t c12 = g1 - g2 + kTop, c13 = g1 - g3 + kTop, c23 = g2 - g3 + kTop;
+  auto maj = [](uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); };
+  const uint32_t k0 = maj(c01, c02, c03);      // kept: beaten at most once
+  const uint32_t k1 = maj(~c01, c12, c13);
+  const uint32_t k2 = maj(~c02, ~c12, c23);
+  const uint32_t k3 = maj(~c03, ~c13, ~c23);
+  // nibble bits: i0 = 0 | 1 | 2 (first kept), i1 = 1 | 2 | 3 (last kept)
+  const uint32_t b0 = ~k0 & k1 & kTop;          // i0 bit 0
+  const uint32_t b1 = ~k0 & ~k1 & kTop;         // i0 bit 1
+  const uint32_t b2 = (k3 | ~k2) & kTop;        // i1 bit 0
+  const uint32_t b3 = (k3 | k2) & kTop;         // i1 bit 1
+  // i0 and i1 of group 0 in bits 0-1 and 8-9, of group 1 in bits 16-17 and
+  // 24-25
+  const uint32_t sp = (b0 >> 15) | (b1 >> 14) | (b2 >> 7) | (b3 >> 6);
+  // nibbles i0 | i1 << 2: group 0 in bits 0-3, group 1 in bits 16-19
+  const uint32_t nib = sp | (sp >> 6);
+  meta = (nib & 0xFu) | ((nib >> 12) & 0xF0u);
+  // kept bf16 values of each group in position order (halfwords i0 and i1):
+  // byte selector 2i0 | (2i0 + 1) << 4 | 2i1 << 8 | (2i1 + 1) << 12, of which
+  // prmt reads only the low 16 bits
+  const uint32_t p0 = prmt(v.x, v.y, sp * 0x22u + 0x1010u);
+  const uint32_t p1 = prmt(v.z, v.w, (sp >> 16) * 0x22u + 0x1010u);
+  if constexpr (kPruned) {
+    // 0xFFFF over kept halfwords: sign of bit 15 (group 0) or 31 (group 1)
+    // of the kept flags, replicated
+    pruned = make_uint4(v.x & prmt(k0, k1, 0xDD99u), v.y & prmt(k2, k3, 0xDD99u),
+                        v.z & prmt(k0, k1, 0xFFBBu), v.w & prmt(k2, k3, 0xFFBBu));
   }
-  // pruned weights: keep positions i0, i1 of each group, +0 elsewhere
-  const uint64_t m0 = (0xFFFFull << (16 * (n0 & 3u))) | (0xFFFFull << (16 * (n0 >> 2)));
-  const uint64_t m1 = (0xFFFFull << (16 * (n1 & 3u))) | (0xFFFFull << (16 * (n1 >> 2)));
-  const uint64_t p0 = g0 & m0, p1 = g1 & m1;
-  pruned = make_uint4(static_cast<uint32_t>(p0), static_cast<uint32_t>(p0 >> 32),
-                      static_cast<uint32_t>(p1), static_cast<uint32_t>(p1 >> 32));
-  return packed;
+  if (d.s == 0.0f) return zero_codes4(p0, p1);
+  return d.codes4(p0, p1);
 }
 
 template <QMode kMode>
@@ -108,8 +118,25 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
   const int t = threadIdx.x;
   const int chunk = t & 15;
-  const int64_t KB = a.K / 128;
+  const int KB = static_cast<int>(a.K / 128);
+  // Tile index = rb * KB + kb; this CTA walks tiles blockIdx.x + j * gridDim.x.
+  // The (rb, kb) of the current tile and of the next tile to load are
+  // stepped without divisions.
+  struct Cursor {
+    int rb, kb;
+  };
+  const int step_rb = static_cast<int>(gridDim.x) / KB, step_kb = static_cast<int>(gridDim.x) % KB;
+  auto advance = [&](Cursor& c) {
+    c.kb += step_kb;
+    c.rb += step_rb;
+    if (c.kb >= KB) {
+      c.kb -= KB;
+      ++c.rb;
+    }
+  };
   const int64_t first = blockIdx.x, step = gridDim.x;
+  Cursor cur{static_cast<int>(blockIdx.x) / KB, static_cast<int>(blockIdx.x) % KB};
+  Cursor load = cur;
 
   if (t == 0) {
     for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
@@ -128,17 +155,17 @@ __global__ void __launch_bounds__(kQThreads, 2)
       const int64_t tile = first + s * step;
       if (tile >= a.num_tiles) break;
       mbar_arrive_expect_tx(&full[s], kTileBytes);
-      tma_load_2d(smem + s * kTileBytes, &tmap_x, &full[s], static_cast<int32_t>((tile % KB) * 128),
-                  static_cast<int32_t>((tile / KB) * 128));
+      tma_load_2d(smem + s * kTileBytes, &tmap_x, &full[s], load.kb * 128, load.rb * 128);
+      advance(load);
       ++issued;
     }
   }
 
   int it = 0;
-  for (int64_t tile = first; tile < a.num_tiles; tile += step, ++it) {
+  for (int64_t tile = first; tile < a.num_tiles; tile += step, ++it, advance(cur)) {
     const int s = it % kQStages;
     const uint32_t parity = static_cast<uint32_t>(it / kQStages) & 1u;
-    const int64_t kb = tile % KB, rb = tile / KB;
+    const int64_t kb = cur.kb, rb = cur.rb;
     if (!mbar_wait(&full[s], parity, a.wait_limit)) {
       record_device_error(a.err, FP8BS_ERR_DEVICE_TIMEOUT);
       *abort_flag = 1;
@@ -152,8 +179,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
     float m = 0.0f;
     if constexpr (kMode != QMode::kAct) {
+      uint32_t m2 = absmax8(v[0]);
 #pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) m = fmaxf(m, amax8(v[i]));
+      for (int i = 1; i < kRowsPerThread; ++i) m2 = bf16x2_absmax(m2, absmax8(v[i]));
+      m = absmax_to_float(m2);
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       if ((t & 31) == 0) red[(it & 1) * kQWarps + (t >> 5)] = m;
@@ -167,8 +196,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
       const int64_t nt = tile + kQStages * step;
       if (nt < a.num_tiles) {
         mbar_arrive_expect_tx(&full[s], kTileBytes);
-        tma_load_2d(smem + s * kTileBytes, &tmap_x, &full[s], static_cast<int32_t>((nt % KB) * 128),
-                    static_cast<int32_t>((nt / KB) * 128));
+        tma_load_2d(smem + s * kTileBytes, &tmap_x, &full[s], load.kb * 128, load.rb * 128);
+        advance(load);
         ++issued;
       }
     }
@@ -177,11 +206,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
       // one 1x128 group per row: 16 threads hold a row
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
-        float rm = amax8(v[i]);
+        float rm = absmax_to_float(absmax8(v[i]));
 #pragma unroll
         for (int off = 8; off >= 1; off >>= 1) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, off));
         const int64_t r = rb * 128 + i * (kQThreads / 16) + (t >> 4);
-        const float sc = __fdiv_rn(rm, 448.0f);
+        const float sc = scale_of_amax(rm);
         if (r < a.rows) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], ScaleDivider(sc));
           if (chunk == 0) a.scale[r * KB + kb] = sc;
@@ -191,7 +220,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
       m = red[(it & 1) * kQWarps];
 #pragma unroll
       for (int w = 1; w < kQWarps; ++w) m = fmaxf(m, red[(it & 1) * kQWarps + w]);
-      const float sc = __fdiv_rn(m, 448.0f);
+      const float sc = scale_of_amax(m);
       if (t == 0) a.scale[rb * KB + kb] = sc;
       const ScaleDivider d(sc);
 #pragma unroll
@@ -201,14 +230,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
         if constexpr (kMode == QMode::kWeight) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], d);
         } else {
-          uint32_t nib2;
+          constexpr bool kOut = kMode == QMode::kPruneOut;
+          uint32_t meta;
           uint4 pr;
-          const uint32_t packed = prune8(v[i], d, nib2, pr);
+          const uint32_t packed = prune8<kOut>(v[i], d, meta, pr);
           // row r: 64 value bytes and 16 metadata bytes per 128-wide K-block
           reinterpret_cast<uint32_t*>(a.q + r * (a.K / 2) + kb * 64)[chunk] = packed;
-          a.meta[r * (a.K / 8) + kb * 16 + chunk] = static_cast<uint8_t>(nib2);
-          if (a.pruned != nullptr)
-            reinterpret_cast<uint4*>(a.pruned + r * a.K + kb * 128)[chunk] = pr;
+          a.meta[r * (a.K / 8) + kb * 16 + chunk] = static_cast<uint8_t>(meta);
+          if constexpr (kOut) reinterpret_cast<uint4*>(a.pruned + r * a.K + kb * 128)[chunk] = pr;
         }
       }
     }
@@ -283,7 +312,8 @@ cudaError_t launch_prune24_compress(const void* w, int64_t N, int64_t K, void* v
   a.meta = meta;
   a.scale = sw;
   a.pruned = static_cast<__nv_bfloat16*>(w_pruned);
-  return launch_stream<QMode::kPrune>(w, N, K, a, stream);
+  return w_pruned != nullptr ? launch_stream<QMode::kPruneOut>(w, N, K, a, stream)
+                             : launch_stream<QMode::kPrune>(w, N, K, a, stream);
 }
 
 }  // namespace fp8bs

@@ -2,7 +2,8 @@
 // CUDA's IEEE division __fdiv_rn, over the whole domain the quantizers use:
 // s = fl32(amax / 448) for every positive finite bf16 amax, and every finite
 // bf16 x with |x| <= amax (both signs). Also checks the E4M3 codes, both of
-// the checked quotient and of the quantizers' branch-free pair path.
+// the checked quotient and of the quantizers' branch-free pair path (both
+// halves of the pair), and the quantizers' scale amax / 448 for every amax.
 #include <cstdint>
 
 #include "../../fp8_block_scaled_group128_b200/csrc/e4m3_codec.cuh"
@@ -24,6 +25,11 @@ __global__ void div_check_kernel(Result* res) {
   const float s = __fdiv_rn(amax, 448.0f);
   const fp8bs::ScaleDivider d(s);
   unsigned long long n = 0, bad_q = 0, bad_c = 0;
+  // the quantizers' scale amax / 448 (and the zero amax, once)
+  if (threadIdx.x == 0) {
+    bad_q += __float_as_uint(fp8bs::scale_of_amax(amax)) != __float_as_uint(s);
+    if (blockIdx.x == 0) bad_q += __float_as_uint(fp8bs::scale_of_amax(0.0f)) != 0u;
+  }
   for (uint32_t xb = threadIdx.x; xb < 0x10000u; xb += blockDim.x) {
     if ((xb & 0x7FFFu) > amax_bits) continue;   // |x| <= amax (same ordering as bits)
     const float x = __uint_as_float(xb << 16);
@@ -39,7 +45,14 @@ __global__ void div_check_kernel(Result* res) {
     const uint32_t c_ref = __nv_cvt_float_to_fp8(q_ref, __NV_SATFINITE, __NV_E4M3);
     // the quantizers' pair path (x in the low half, +0 in the high half)
     const uint32_t c2 = d.codes2(xb) & 0xFFu;
-    bad_c += (c != c_ref) + (c2 != c_ref);
+    // both halves: x in the high half, -x in the low half
+    const uint32_t c2p = d.codes2((xb << 16) | (xb ^ 0x8000u));
+    // four at once: (x, -x) in the first word, (-x, x) in the second
+    const uint32_t c4 = d.codes4((xb << 16) | (xb ^ 0x8000u), ((xb ^ 0x8000u) << 16) | xb);
+    bad_c += (c4 != (c2p | ((((c2p & 0xFFu) << 8) | (c2p >> 8)) << 16)));
+    const uint32_t cn_ref =
+        __nv_cvt_float_to_fp8(__fdiv_rn(-x, s), __NV_SATFINITE, __NV_E4M3);
+    bad_c += (c != c_ref) + (c2 != c_ref) + ((c2p >> 8) != c_ref) + ((c2p & 0xFFu) != cn_ref);
   }
   atomicAdd(&res->checked, n);
   if (bad_q) atomicAdd(&res->quotient_mismatch, bad_q);

@@ -147,3 +147,35 @@ def test_prune_sparse_config_sampled_blocks(N, K):
     NB = -(-N // 128)
     blocks = sorted(set([0, NB - 1] + list(np.random.default_rng(K).choice(NB, 4, replace=False))))
     _prune_case(w, row_blocks=blocks)
+
+
+def _all_patterns_matrix():
+    """Rows of 256 groups of 4 covering every assignment of 4 magnitude levels
+    to the 4 positions of a group (4^4 patterns, so every tie structure), for
+    three level sets: small multiples of 0.25, adjacent bf16 values, and the
+    extremes of the bf16 magnitude range (0, smallest subnormal, the two
+    largest finite values). Signs are random per element."""
+    levels = [np.array([0x0000, 0x3E80, 0x3F00, 0x3F40], np.uint16),   # 0, .25, .5, .75
+              np.array([0x3F80, 0x3F81, 0x3F82, 0x3F83], np.uint16),   # adjacent bf16
+              np.array([0x0000, 0x0001, 0x7F7E, 0x7F7F], np.uint16)]   # range ends
+    idx = np.array(np.meshgrid(*[np.arange(4)] * 4, indexing="ij")).reshape(4, -1).T  # [256, 4]
+    rng = np.random.default_rng(11)
+    rows = []
+    for lv in levels:
+        for r in range(128):
+            perm = np.roll(idx, r, axis=0)               # each row holds every pattern
+            bits = lv[perm].reshape(-1)
+            sign = rng.integers(0, 2, size=bits.shape).astype(np.uint16) << 15
+            rows.append(bits | sign)
+    return torch.from_numpy(np.stack(rows).view(np.int16)).view(torch.bfloat16)
+
+
+def test_prune_every_tie_pattern():
+    w = _all_patterns_matrix()                      # [384, 1024]
+    _prune_case(w)
+    # the path without the pruned output writes the same bytes
+    a = fb.prune24_compress(to_dev(w), want_pruned=True)
+    b = fb.prune24_compress(to_dev(w))
+    torch.cuda.synchronize()
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))

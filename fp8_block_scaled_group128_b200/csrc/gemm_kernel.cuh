@@ -48,6 +48,7 @@ namespace gemm_detail {
 constexpr int kBK = 128;               // K-block depth = one scale group, 128 bytes of E4M3
 constexpr int kGroupRows = 16;         // tile raster: row tiles per group (L2 reuse)
 constexpr int kEBytes = 128 * 16;      // sparse: metadata of one 128x128 block, 16 B per row
+constexpr int kG = 8;                  // K-blocks per group of the epilogue's scale table
 
 struct GemmArgs {
   const float* sa;      // [M][KB]
@@ -96,10 +97,17 @@ struct Cfg {
   static constexpr int kNumBars = 2 * kStages + 2 * kBufs + 1;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmem + 4;
-  // decode: per-epilogue-warp column scales of the current K-block
-  static constexpr int kOffScr = (kOffAbort + 4 + 15) / 16 * 16;
-  static constexpr int kScrBytes = kSwap ? 4 * kEpiWG * kCols * 4 : 0;
-  static constexpr int kSmemBytes = kOffScr + kScrBytes + 1024;  // + slack to align the base
+  // scale table of the epilogue: 2 buffers x kG K-blocks x kSlots token
+  // slots (row stride padded by 4 floats: conflict-free transposed stores,
+  // 16-byte aligned rows)
+  static constexpr int kEpiThreads = 128 * kEpiWG;
+  static constexpr int kSlots = kSwap ? BN : 128 * kEpiWG;
+  static constexpr int kTabStride = kSlots + 4;
+  static constexpr int kPer = kG * kSlots / kEpiThreads;   // staged values per thread
+  static_assert(kG * kSlots % kEpiThreads == 0, "scale table split");
+  static constexpr int kOffTab = (kOffAbort + 4 + 15) / 16 * 16;
+  static constexpr int kTabBytes = 2 * kG * kTabStride * 4;
+  static constexpr int kSmemBytes = kOffTab + kTabBytes + 1024;  // + slack to align the base
   // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
   static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -316,75 +324,102 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     const int quarter = warp & 3;       // TMEM lanes [32 quarter, 32 quarter + 32)
     const int row = quarter * 32 + lane;
     const int col0 = wg * C::kCols;
-    const int KB = args.KB;
-    float* scr = reinterpret_cast<float*>(smem + C::kOffScr) + (warp - 4) * C::kCols;
+    const int64_t KB = args.KB;
+    const int e = static_cast<int>(threadIdx.x) - 128;   // epilogue thread index
+    float* tab = reinterpret_cast<float*>(smem + C::kOffTab);
+
+    // Scale table. Every element of a K-block partial is scaled by
+    // sA[token, kb] * sW[weight row block, kb]. Per group of kG K-blocks the
+    // epilogue warps stage these products for every token slot of the tile in
+    // a double-buffered shared table [kG][kSlots] (global loads run along kb,
+    // one group ahead of its use), and the promotion reads them from shared
+    // memory. Slots: decode order = the BN token columns; prefill order = the
+    // 128 token rows, once per epilogue warpgroup (each has its own weight
+    // block). The groups of this CTA are (tile, kbg) for its tiles in order and
+    // kbg = kb0, kb0 + kG, ... < kb1.
+    int g_tile = blockIdx.y, g_kb = kb0;   // next group to stage
+    // raw loads of the next group; multiplied only when stored, a group
+    // later, so that nothing waits on them
+    float pre_a[C::kPer], pre_w[C::kPer];
+    auto group_load = [&]() {
+      if (g_tile >= num_tiles) return;
+      int grt, gct;
+      tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
+#pragma unroll
+      for (int i = 0; i < C::kPer; ++i) {
+        const int idx = e + C::kEpiThreads * i;
+        const int g = idx % kG, slot = idx / kG;
+        const int kb = g_kb + g;
+        float va = 0.0f, vw = 0.0f;
+        if (kb < kb1) {
+          if constexpr (kSwap) {
+            const int64_t tok = static_cast<int64_t>(gct) * BN + slot;
+            if (tok < args.M) {
+              va = args.sa[tok * KB + kb];
+              vw = args.sw[grt * KB + kb];
+            }
+          } else {
+            const int64_t m = static_cast<int64_t>(grt) * 128 + (slot & 127);
+            const int nb = (gct * BN + (slot >> 7) * C::kCols) / 128;
+            if (m < args.M && nb < args.NB) {
+              va = args.sa[m * KB + kb];
+              vw = args.sw[nb * KB + kb];
+            }
+          }
+        }
+        pre_a[i] = va;
+        pre_w[i] = vw;
+      }
+    };
+    auto group_store = [&](int buf) {
+#pragma unroll
+      for (int i = 0; i < C::kPer; ++i) {
+        const int idx = e + C::kEpiThreads * i;
+        tab[(buf * kG + idx % kG) * C::kTabStride + idx / kG] = pre_a[i] * pre_w[i];
+      }
+    };
+    auto group_next = [&]() {
+      g_kb += kG;
+      if (g_kb >= kb1) {
+        g_kb = kb0;
+        g_tile += gridDim.y;
+      }
+    };
+    group_load();
+    group_store(0);
+    group_next();
+    group_load();
+    named_bar_sync(1, C::kEpiThreads);
+    int buf = 0;
+
     int tb = 0;
     uint32_t tphase = 0;
     bool ok = true;
-    for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+    // Every epilogue thread walks the same groups (the named barrier above
+    // needs all of them); after a wait runs out, `ok` is false and the rest is
+    // skipped.
+    for (int tile = blockIdx.y; tile < num_tiles; tile += gridDim.y) {
       int rt, ct;
       tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
 #pragma unroll
       for (int i = 0; i < C::kCols; ++i) acc[i] = 0.0f;
 
-      // Scale sources. Prefill: one scale per thread and K-block,
-      // sA[m,kb] * sW[nb,kb]. Decode (swap): one scale per column (token),
-      // sW[rt,kb] * sA[tok,kb]; lane l fetches the scale of column (32c + l)
-      // of each 32-column chunk c and the warp shares them by shuffles.
-      const int m = rt * 128 + row;
-      const int nb = (ct * BN + col0) / 128;
-      const float* sa_row = args.sa + static_cast<int64_t>(m < args.M ? m : 0) * KB;
-      const bool row_ok = !kSwap && m < args.M && nb < args.NB;
-      constexpr int kChunks = C::kCols / 32 > 0 ? C::kCols / 32 : 1;
-      int tok_l[kChunks];
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) tok_l[c] = ct * BN + col0 + 32 * c + lane;
-
-      // The loads land in the ring untouched (the product is formed only when
-      // the K-block is consumed, so nothing waits on a load early).
-      auto load_scales = [&](int kb, float* sa_v, float& sw_v) {
-        if constexpr (!kSwap) {
-          sa_v[0] = row_ok ? sa_row[kb] : 0.0f;
-          sw_v = row_ok ? args.sw[static_cast<int64_t>(nb) * KB + kb] : 0.0f;
-        } else {
-          sw_v = args.sw[static_cast<int64_t>(rt) * KB + kb];
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            const bool tok_ok = tok_l[c] < args.M && (32 * c + lane) < C::kCols;
-            sa_v[c] = tok_ok ? args.sa[static_cast<int64_t>(tok_l[c]) * KB + kb] : 0.0f;
-          }
-        }
-      };
-      // Scales are prefetched kPrefetch K-blocks ahead into a register ring
-      // indexed at compile time (the K loop is unrolled by kPrefetch).
-      constexpr int kPrefetch = 4;
-      float ring_a[kPrefetch][kChunks];
-      float ring_w[kPrefetch];
-#pragma unroll
-      for (int d = 0; d < kPrefetch; ++d)
-        if (kb0 + d < kb1) load_scales(kb0 + d, ring_a[d], ring_w[d]);
-
-      for (int kb_base = kb0; ok && kb_base < kb1; kb_base += kPrefetch) {
-#pragma unroll
-        for (int d = 0; d < kPrefetch; ++d) {
-          const int kb = kb_base + d;
-          if (!ok || kb >= kb1) break;
+      for (int kbg = kb0; kbg < kb1; kbg += kG) {
+        const float* tg = tab + buf * kG * C::kTabStride;
+        for (int j = 0; ok && j < kG; ++j) {
+          const int kb = kbg + j;
+          if (kb >= kb1) break;
           if (!mbar_wait(&tfull[tb], tphase, limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if constexpr (kSwap) {
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c)
-              if (32 * c + lane < C::kCols) scr[32 * c + lane] = ring_w[d] * ring_a[d][c];
-            __syncwarp();
-          }
+          const float* trow = tg + j * C::kTabStride;
           const uint32_t taddr =
               tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
           if constexpr (!kSwap && C::kCols % 64 == 0) {
             // prefill: 64 columns per TMEM round trip (two x32 loads, one wait)
-            const float sc = ring_a[d][0] * ring_w[d];
+            const float sc = trow[wg * 128 + row];
 #pragma unroll
             for (int c = 0; c < C::kCols; c += 64) {
               float v[64];
@@ -403,7 +438,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
             if (c + 16 < C::kCols) tmem_ld16(taddr + c + 16, v1);
             tmem_wait_ld();
             if constexpr (!kSwap) {
-              const float sc = ring_a[d][0] * ring_w[d];
+              const float sc = trow[wg * 128 + row];
 #pragma unroll
               for (int i = 0; i < 16; ++i) acc[c + i] = fmaf(sc, v0[i], acc[c + i]);
               if (c + 16 < C::kCols) {
@@ -411,8 +446,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
                 for (int i = 0; i < 16; ++i) acc[c + 16 + i] = fmaf(sc, v1[i], acc[c + 16 + i]);
               }
             } else {
-              // column scales of this K-block, broadcast from the warp's slot
-              const float4* s4 = reinterpret_cast<const float4*>(scr + c);
+              // column scales of this K-block (the same for every lane)
+              const float4* s4 = reinterpret_cast<const float4*>(trow + col0 + c);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const float4 q = s4[i];
@@ -432,20 +467,26 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
             }
           }
           tc_fence_before();
-          __syncwarp();   // also: every lane is done reading this K-block's scales
+          __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[tb]);
           if (++tb == C::kBufs) {
             tb = 0;
             tphase ^= 1u;
           }
-          if (kb + kPrefetch < kb1) load_scales(kb + kPrefetch, ring_a[d], ring_w[d]);
         }
+        // the group after this one goes into the other buffer (nobody reads it
+        // any more: its last readers passed the previous barrier)
+        group_store(buf ^ 1);
+        group_next();
+        group_load();
+        named_bar_sync(1, C::kEpiThreads);
+        buf ^= 1;
       }
-      if (!ok) break;
 
-      if (args.splits == 1) {
+      if (ok && args.splits == 1) {
         if constexpr (!kSwap) {
           // row m of Y, columns [n0, n0 + kCols): 16-byte stores of 8 bf16
+          const int m = rt * 128 + row;
           const int n0 = ct * BN + col0;
           if (m < args.M) {
             __nv_bfloat16* yrow = args.y + static_cast<int64_t>(m) * args.N;

@@ -36,7 +36,9 @@
 // flight, frees TMEM and returns.
 #pragma once
 
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -107,7 +109,11 @@ struct Cfg {
   static_assert(kG * kSlots % kEpiThreads == 0, "scale table split");
   static constexpr int kOffTab = (kOffAbort + 4 + 15) / 16 * 16;
   static constexpr int kTabBytes = 2 * kG * kTabStride * 4;
-  static constexpr int kSmemBytes = kOffTab + kTabBytes + 1024;  // + slack to align the base
+  // prefill: the bf16 output tile [128][BN], staged for TMA stores as boxes
+  // of 128 rows x 64 columns (128 bytes, 128-byte swizzle), 16 KB each
+  static constexpr int kOffOut = (kOffTab + kTabBytes + 1023) / 1024 * 1024;
+  static constexpr int kOutBytes = kSwap ? 0 : 128 * BN * 2;
+  static constexpr int kSmemBytes = kOffOut + kOutBytes + 1024;  // + slack to align the base
   // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
   static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -135,8 +141,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_e, const GemmArgs args) {
+  // tmap_e: the 2:4 metadata (sparse) or the output Y (prefill order)
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
-  constexpr int kABytes = C::kABytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -483,38 +489,54 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
         buf ^= 1;
       }
 
-      if (ok && args.splits == 1) {
-        if constexpr (!kSwap) {
-          // row m of Y, columns [n0, n0 + kCols): 16-byte stores of 8 bf16
-          const int m = rt * 128 + row;
-          const int n0 = ct * BN + col0;
-          if (m < args.M) {
-            __nv_bfloat16* yrow = args.y + static_cast<int64_t>(m) * args.N;
+      if constexpr (!kSwap) {
+        // This warpgroup's 128 columns = two 64-column boxes of the staged
+        // tile. Its leader first waits until the previous tile's stores have
+        // read the boxes; every thread then writes its row (16-byte chunk j
+        // of row r at chunk position j ^ (r % 8): the 128-byte swizzle), and
+        // the leader issues the two TMA stores, which run on while the next
+        // tile is promoted. TMA leaves rows >= M and columns >= N unwritten.
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        uint8_t* out = smem + C::kOffOut + wg * (C::kCols / 64) * 16384;
+        if (leader) bulk_wait_group_read0();
+        named_bar_sync(2 + wg, 128);
+        if (ok) {
 #pragma unroll
-            for (int c = 0; c < C::kCols; c += 8) {
-              if (n0 + c < args.N) {
-                uint4 pk;
-                pk.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
-                pk.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
-                pk.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
-                pk.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
-                *reinterpret_cast<uint4*>(yrow + n0 + c) = pk;
-              }
-            }
+          for (int c = 0; c < C::kCols; c += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(acc[c + 0], acc[c + 1]);
+            pk.y = pack_bf16x2(acc[c + 2], acc[c + 3]);
+            pk.z = pack_bf16x2(acc[c + 4], acc[c + 5]);
+            pk.w = pack_bf16x2(acc[c + 6], acc[c + 7]);
+            const int j = (c & 63) >> 3;
+            *reinterpret_cast<uint4*>(out + (c >> 6) * 16384 + row * 128 +
+                                      ((j ^ (row & 7)) << 4)) = pk;
           }
-        } else {
-          // column j of the tile is token ct*BN + col0 + j; row is weight row n
-          const int n = rt * 128 + row;
-          if (n < args.N) {
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2 + wg, 128);
+        if (leader && ok) {
 #pragma unroll
-            for (int j = 0; j < C::kCols; ++j) {
-              const int tok = ct * BN + col0 + j;
-              if (tok < args.M)
-                args.y[static_cast<int64_t>(tok) * args.N + n] = __float2bfloat16_rn(acc[j]);
-            }
+          for (int b = 0; b < C::kCols / 64; ++b)
+            tma_store_2d(&tmap_e, out + b * 16384, ct * BN + col0 + b * 64, rt * 128);
+          bulk_commit_group();
+        }
+      } else if (ok && args.splits == 1) {
+        // column j of the tile is token ct*BN + col0 + j; row is weight row n
+        const int n = rt * 128 + row;
+        if (n < args.N) {
+#pragma unroll
+          for (int j = 0; j < C::kCols; ++j) {
+            const int tok = ct * BN + col0 + j;
+            if (tok < args.M)
+              args.y[static_cast<int64_t>(tok) * args.N + n] = __float2bfloat16_rn(acc[j]);
           }
         }
       }
+    }
+    // prefill: the last stores have finished before the CTA exits
+    if constexpr (!kSwap) {
+      if ((warp & 3) == 0 && lane == 0) bulk_wait_group0();
     }
     if (!ok) {
       record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
@@ -597,28 +619,30 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
 // kernel, device and S).
 template <class Kern>
 int max_active_clusters(Kern kern, int threads, int smem, int S, int dev) {
-  static int cache[64][9];
-  static std::once_flag flags[64][9];
-  std::call_once(flags[dev][S], [&] {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
-    cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = static_cast<unsigned>(S);
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
-    }
-    cache[dev][S] = n;
-  });
-  return cache[dev][S];
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int>, int> cache;
+  const auto key = std::make_tuple(reinterpret_cast<const void*>(kern), dev, S);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = static_cast<unsigned>(S);
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;   // not cached: a later call may succeed
+  }
+  cache[key] = n;
+  return n;
 }
 
 template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>

@@ -195,8 +195,20 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Set-up above touches no global memory; inputs may come from the previous
-  // kernel of the stream.
+  // Dense decode order: the weight stages of the first tile are prefetched
+  // into L2 while the previous kernel of the stream may still run (an L2
+  // prefetch never changes what a later load reads, so this is safe even if
+  // that kernel writes the weights). Measured: 3-7 % faster dense decode
+  // launches; the 2:4 launches ran slower with it, so they do without.
+  if constexpr (kSwap && !kSparse) {
+    if (threadIdx.x == 0 && static_cast<int>(blockIdx.y) < num_tiles) {
+      int rt, ct;
+      tile_coords(blockIdx.y, args.row_tiles, args.col_tiles, rt, ct);
+      for (int kb = kb0, n = 0; kb < kb1 && n < kStages; kb += kKS, ++n)
+        tma_prefetch_l2_3d(&tmap_a, 0, rt * 128, kb);
+    }
+  }
+  // Everything else waits: inputs may come from the previous kernel.
   grid_dependency_wait();
   grid_launch_dependents();
 

@@ -1,5 +1,5 @@
-// Streaming quantizers over 128x128 bf16 tiles: activation groups (S1),
-// weight blocks (S2) and 2:4 prune + compress (S4).
+// The quantizers: activation groups (S1, act_quant_kernel), and, streaming
+// 128x128 bf16 tiles, weight blocks (S2) and 2:4 prune + compress (S4).
 //
 // Rules: "FP8 à granularité fine", opening bullets (one fp32 scale per 1x128
 // group of a token, or per 128x128 weight block; s = amax / 448, code =
@@ -9,7 +9,7 @@
 // two largest |w| of each 4 along K, ties to the lower index, pruned -> +0;
 // scales from the pruned block).
 //
-// All three are HBM streaming kernels. CTAs are persistent (two per SM); thread
+// The tile kernel (S2, S4) streams HBM. CTAs are persistent (two per SM); thread
 // 0 keeps a 3-deep ring of 32 KB tiles in flight with TMA
 // (cp.async.bulk.tensor, no swizzle, out-of-range rows read as zero), and all
 // 512 threads work from shared memory. Thread t owns the 16-byte chunk t % 16
@@ -27,7 +27,7 @@ namespace fp8bs {
 namespace {
 
 // kPruneOut: 2:4 prune + compress that also writes the pruned bf16 weights.
-enum class QMode { kAct, kWeight, kPrune, kPruneOut };
+enum class QMode { kWeight, kPrune, kPruneOut };
 
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
@@ -177,8 +177,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
       v[i] = *reinterpret_cast<const uint4*>(buf + (i * (kQThreads / 16) + (t >> 4)) * 256 +
                                              chunk * 16);
 
-    float m = 0.0f;
-    if constexpr (kMode != QMode::kAct) {
+    float m;
+    {
       uint32_t m2 = absmax8(v[0]);
 #pragma unroll
       for (int i = 1; i < kRowsPerThread; ++i) m2 = bf16x2_absmax(m2, absmax8(v[i]));
@@ -202,21 +202,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
       }
     }
 
-    if constexpr (kMode == QMode::kAct) {
-      // one 1x128 group per row: 16 threads hold a row
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        float rm = absmax_to_float(absmax8(v[i]));
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, off));
-        const int64_t r = rb * 128 + i * (kQThreads / 16) + (t >> 4);
-        const float sc = scale_of_amax(rm);
-        if (r < a.rows) {
-          reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], ScaleDivider(sc));
-          if (chunk == 0) a.scale[r * KB + kb] = sc;
-        }
-      }
-    } else {
+    {
       m = red[(it & 1) * kQWarps];
 #pragma unroll
       for (int w = 1; w < kQWarps; ++w) m = fmaxf(m, red[(it & 1) * kQWarps + w]);
@@ -286,14 +272,74 @@ cudaError_t launch_stream(const void* x, int64_t rows, int64_t K, QArgs a, cudaS
   return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
+// Activation quantization (S1). A team of 16 threads quantizes 1x128
+// groups: each thread one 16-byte chunk (8 bf16) of a group, a 16-lane
+// shuffle max, the encode of e4m3_codec.cuh, one 8-byte store; the team's
+// first thread writes the scale. A team takes kGroups groups spread over the
+// grid (team, team + teams, ...) and issues all their loads before any
+// arithmetic: 4 for inputs that fill the GPU many times over (64 bytes per
+// thread in flight), 1 for decode-sized inputs (lowest latency). Groups are
+// contiguous in memory (row-major [M][K], K a multiple of 128) and the scale
+// of group g is sa[g] (row-major [M][K/128]). No shared memory and no
+// barrier: for decode-sized inputs the kernel costs one load round trip.
+constexpr int kActThreads = 256;
+
+template <int kGroups>
+__global__ void __launch_bounds__(kActThreads)
+    act_quant_kernel(const __nv_bfloat16* __restrict__ x, int64_t groups,
+                     uint8_t* __restrict__ q, float* __restrict__ scale) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t teams = static_cast<int64_t>(gridDim.x) * (kActThreads / 16);
+  const int64_t team = static_cast<int64_t>(blockIdx.x) * (kActThreads / 16) + (threadIdx.x >> 4);
+  const int chunk = threadIdx.x & 15;
+  uint4 v[kGroups];
+#pragma unroll
+  for (int j = 0; j < kGroups; ++j) {
+    const int64_t g = team + j * teams;
+    v[j] = g < groups ? __ldg(reinterpret_cast<const uint4*>(x + g * 128) + chunk)
+                      : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int j = 0; j < kGroups; ++j) {
+    const int64_t g = team + j * teams;
+    float m = absmax_to_float(absmax8(v[j]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float sc = scale_of_amax(m);
+    if (g < groups) {
+      reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8(v[j], ScaleDivider(sc));
+      if (chunk == 0) scale[g] = sc;
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_act_group128(const void* x, int64_t M, int64_t K, void* qa, float* sa,
                                       cudaStream_t stream) {
-  QArgs a{};
-  a.q = static_cast<uint8_t*>(qa);
-  a.scale = sa;
-  return launch_stream<QMode::kAct>(x, M, K, a, stream);
+  DeviceInfo dev;
+  if (current_device_info(&dev) != FP8BS_OK) return cudaErrorInvalidDevice;
+  const int64_t groups = M * (K / 128);
+  const int64_t teams_per_block = kActThreads / 16;
+  // one group per team unless one team per group would fill every SM
+  // (2048 threads) eight times over
+  const int per = groups >= 8LL * dev.sm_count * (2048 / 16) ? 4 : 1;
+  const int64_t blocks = (groups + teams_per_block * per - 1) / (teams_per_block * per);
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(kActThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  auto* qp = static_cast<uint8_t*>(qa);
+  return per == 4 ? cudaLaunchKernelEx(&cfg, act_quant_kernel<4>, xp, groups, qp, sa)
+                  : cudaLaunchKernelEx(&cfg, act_quant_kernel<1>, xp, groups, qp, sa);
 }
 
 cudaError_t launch_quant_weight_block128(const void* w, int64_t N, int64_t K, void* qw, float* sw,

@@ -49,7 +49,7 @@ def test_act_quant_prefill_shapes_sampled_rows(M, K):
     _act_case(x, rows=rows)
 
 
-@pytest.mark.parametrize("M", [3, 5, 33, 257])
+@pytest.mark.parametrize("M", [3, 5, 33, 256, 257])
 def test_act_quant_ragged_group_counts(M):
     # M * K / 128 not a multiple of 4: the last warp's unit is partial
     _act_case(synth.activations("deepseek", M, 384, seed=M))

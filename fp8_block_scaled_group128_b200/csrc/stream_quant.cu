@@ -32,9 +32,8 @@ enum class QMode { kWeight, kPrune, kPruneOut };
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
 constexpr int kQThreads = 512;
-constexpr int kQWarps = kQThreads / 32;
 constexpr int kRowsPerThread = 128 * 16 / kQThreads;   // 16 threads per 256-byte row
-constexpr int kQSmemBytes = kQStages * kTileBytes + 1024 + 512;
+constexpr int kQSmemBytes = kQStages * kTileBytes + 1024 + 64;
 
 struct QArgs {
   int64_t rows;            // M (activations) or N (weights)
@@ -113,8 +112,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kTileBytes);
-  float* red = reinterpret_cast<float*>(full + kQStages);   // [2][kQWarps] block-max partials
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 2 * kQWarps);
+  // block max of tile `it` in slot it % 3, as the bits of a non-negative
+  // float (ordered like the values): a slot is cleared two tiles ahead, after
+  // everyone has read it
+  unsigned* red = reinterpret_cast<unsigned*>(full + kQStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 4);
 
   const int t = threadIdx.x;
   const int chunk = t & 15;
@@ -140,6 +142,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
   if (t == 0) {
     for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    red[0] = red[1] = red[2] = 0u;
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_x);
@@ -177,15 +180,13 @@ __global__ void __launch_bounds__(kQThreads, 2)
       v[i] = *reinterpret_cast<const uint4*>(buf + (i * (kQThreads / 16) + (t >> 4)) * 256 +
                                              chunk * 16);
 
-    float m;
     {
       uint32_t m2 = absmax8(v[0]);
 #pragma unroll
       for (int i = 1; i < kRowsPerThread; ++i) m2 = bf16x2_absmax(m2, absmax8(v[i]));
-      m = absmax_to_float(m2);
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if ((t & 31) == 0) red[(it & 1) * kQWarps + (t >> 5)] = m;
+      const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(absmax_to_float(m2)));
+      if ((t & 31) == 0) atomicMax(&red[it % 3], mw);
+      if (t == 0) red[(it + 1) % 3] = 0u;   // read by everyone before the previous barrier
     }
     // Every thread has read stage s (and published its block-max partial);
     // the proxy fence orders those reads before the TMA that refills stage s.
@@ -203,16 +204,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
     }
 
     {
-      m = red[(it & 1) * kQWarps];
-#pragma unroll
-      for (int w = 1; w < kQWarps; ++w) m = fmaxf(m, red[(it & 1) * kQWarps + w]);
-      const float sc = scale_of_amax(m);
+      const float sc = scale_of_amax(__uint_as_float(red[it % 3]));
       if (t == 0) a.scale[rb * KB + kb] = sc;
       const ScaleDivider d(sc);
+      // this thread's first row and its outputs; rows i step by kQThreads / 16
+      const int64_t r0 = rb * 128 + (t >> 4);
+      const int rows_here = static_cast<int>(a.rows - r0 < 0 ? 0 : a.rows - r0);
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
-        const int64_t r = rb * 128 + i * (kQThreads / 16) + (t >> 4);
-        if (r >= a.rows) continue;
+        if (i * (kQThreads / 16) >= rows_here) break;
+        const int64_t r = r0 + i * (kQThreads / 16);
         if constexpr (kMode == QMode::kWeight) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], d);
         } else {

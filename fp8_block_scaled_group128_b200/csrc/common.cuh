@@ -64,15 +64,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most
-// `limit` clock cycles. Returns false if the limit ran out.
+// `limit` clock cycles. Returns false if the limit ran out. The first probe
+// does not block, so a limit of a few cycles gives up at once on any phase
+// that is not complete yet.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  for (;;) {
+    // the limit is checked before each (possibly suspending) probe
     if (clock64() - t0 > limit) return false;
+    if (mbar_try_wait(bar, parity)) return true;
   }
-  return true;
+}
+
+// True in exactly one lane of the converged warp (elect.sync). A loop that
+// the whole warp runs, with only its issuing instruction under this
+// predicate, keeps its operands warp-uniform, which makes tcgen05 and TMA
+// issue much cheaper than from a one-lane branch.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // Orders this thread's earlier generic-proxy shared-memory accesses before its
@@ -220,6 +250,19 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
       : "memory");
 }
 
+// The same with the accumulate flag a compile-time constant (no predicate
+// set-up at run time in the MMA issue loop).
+template <bool kAccumulate>
+__device__ __forceinline__ void mma_f8f6f4_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "n"(kAccumulate ? 1 : 0)
+      : "memory");
+}
+
 // 2:4 sparse A: D[tmem] (+)= A[smem desc, compressed] * B[smem desc]^T with
 // the A metadata read from TMEM at `e_tmem` (kind::f8f6f4, one CTA).
 __device__ __forceinline__ void mma_sp_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -230,6 +273,17 @@ __device__ __forceinline__ void mma_sp_f8f6f4(uint32_t d_tmem, uint64_t adesc, u
       "setp.ne.b32 p, %5, 0;\n\t"
       "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <bool kAccumulate>
+__device__ __forceinline__ void mma_sp_f8f6f4_c(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t e_tmem, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "n"(kAccumulate ? 1 : 0)
       : "memory");
 }
 

@@ -224,116 +224,129 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   if (warp < 4) {
    if constexpr (kRegSplit) setmaxnreg_dec<40>();
    if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------ TMA producer --
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      for (int tile = blockIdx.y; tile < num_tiles && !*abort_flag; tile += gridDim.y) {
-        int rt, ct;
-        tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
-        for (int kb = kb0; kb < kb1; kb += kKS) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
-            record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
-            *abort_flag = 1;
-            break;
-          }
-          // one box per operand covers K-blocks [kb, kb + kKS) (K-blocks past
-          // the end of K read as zero and are not used)
+    // -------------------------------------------------------- TMA producer --
+    // The whole warp runs the loop; one elected lane issues.
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    for (int tile = blockIdx.y; tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+      int rt, ct;
+      tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
+      for (int kb = kb0; kb < kb1; kb += kKS) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
+          record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        // one box per operand covers K-blocks [kb, kb + kKS) (K-blocks past
+        // the end of K read as zero and are not used)
+        if (elect_one()) {
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           tma_load_3d(sm_a + stage * C::kABytes, &tmap_a, &full[stage], 0, rt * 128, kb);
           if constexpr (kSparse)
             tma_load_3d(sm_e + stage * C::kEStage, &tmap_e, &full[stage], 0, rt * 128, kb);
           tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, ct * BN, kb);
-          ++issued;
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-      }
-      // Every copy issued must have landed before shared memory is reused or
-      // the CTA exits (matters only when a consumer stopped early).
-      const int pending = issued < kStages ? issued : kStages;
-      for (int i = 0; i < pending; ++i) {
-        int s = stage - 1 - i;
-        uint32_t ph = phase;
-        if (s < 0) {
-          s += kStages;
-          ph ^= 1u;
+        __syncwarp();
+        ++issued;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
         }
-        mbar_wait(&full[s], ph, kDefaultWaitCycles);
       }
     }
+    // Every copy issued must have landed before shared memory is reused or
+    // the CTA exits (matters only when a consumer stopped early).
+    const int pending = issued < kStages ? issued : kStages;
+    for (int i = 0; i < pending; ++i) {
+      int s = stage - 1 - i;
+      uint32_t ph = phase;
+      if (s < 0) {
+        s += kStages;
+        ph ^= 1u;
+      }
+      mbar_wait(&full[s], ph, kDefaultWaitCycles);
+    }
    } else if (warp == 1) {
-    if (lane == 0) {
-      // -------------------------------------------------------- MMA issuer --
-      int stage = 0;
-      uint32_t phase = 0;
-      int tb = 0;
-      uint32_t tphase = 0;
-      uint32_t e_buf = 0;  // sparse: TMEM metadata buffer, alternating per K-block
-      bool ok = true;
-      for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
-        for (int kb = kb0; ok && kb < kb1; kb += kKS) {
-          if (!mbar_wait(&full[stage], phase, limit)) {
+    // ---------------------------------------------------------- MMA issuer --
+    // The whole warp runs the loop (warp-uniform operands); one elected lane
+    // issues each tcgen05 operation.
+    int stage = 0;
+    uint32_t phase = 0;
+    int tb = 0;
+    uint32_t tphase = 0;
+    uint32_t e_buf = 0;  // sparse: TMEM metadata buffer, alternating per K-block
+    bool ok = true;
+    // Shared-memory descriptors of stage 0, K-block 0; every other operand
+    // tile is an offset from them: the start-address field is address >> 4 in
+    // the low 14 bits and shared addresses stay below 2^18, so adding
+    // offset >> 4 moves it without touching the other fields.
+    const uint64_t da0 = kSparse ? sw64_kmajor_desc(smem_u32(sm_a)) : sw128_kmajor_desc(smem_u32(sm_a));
+    const uint64_t db0 = sw128_kmajor_desc(smem_u32(sm_b));
+    const uint64_t de0 = kSparse ? noswizzle_kmajor_desc(smem_u32(sm_e), 128) : 0;
+    for (int tile = blockIdx.y; ok && tile < num_tiles && !*abort_flag; tile += gridDim.y) {
+      for (int kb = kb0; ok && kb < kb1; kb += kKS) {
+        if (!mbar_wait(&full[stage], phase, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < kKS; ++j) {
+          if (kb + j >= kb1) break;
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < kKS; ++j) {
-            if (kb + j >= kb1) break;
-            if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
-              ok = false;
-              break;
+          const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
+          const uint64_t da = da0 + static_cast<uint32_t>((stage * C::kABytes + j * C::kAKb) >> 4);
+          const uint64_t db = db0 + static_cast<uint32_t>((stage * C::kBBytes + j * C::kBKb) >> 4);
+          if constexpr (kSparse) {
+            // metadata of this K-block -> TMEM (4 columns, lane = weight
+            // row), then two sparse MMAs of logical depth 64 (32 compressed
+            // bytes of A and 64 bytes of B each), reading 2 metadata columns
+            const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
+            e_buf ^= 1u;
+            const uint64_t de = de0 + static_cast<uint32_t>((stage * C::kEStage + j * kEBytes) >> 4);
+            if (elect_one()) {
+              tmem_cp_128x128b(te, de);
+              mma_sp_f8f6f4_c<false>(d, da, db, te, C::kIdesc);
+              mma_sp_f8f6f4_c<true>(d, da + (32 >> 4), db + (64 >> 4), te + 2, C::kIdesc);
+              mma_commit(&tfull[tb]);
             }
-            tc_fence_after();
-            const uint32_t d = tmem_base + static_cast<uint32_t>(tb * BN);
-            const uint32_t a0 = smem_u32(sm_a + stage * C::kABytes + j * C::kAKb);
-            const uint32_t b0 = smem_u32(sm_b + stage * C::kBBytes + j * C::kBKb);
-            if constexpr (kSparse) {
-              // metadata of this K-block -> TMEM (4 columns, lane = weight
-              // row), then two sparse MMAs of logical depth 64 (32 compressed
-              // bytes of A and 64 bytes of B each), reading 2 metadata columns
-              const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
-              e_buf ^= 1u;
-              tmem_cp_128x128b(
-                  te, noswizzle_kmajor_desc(smem_u32(sm_e + stage * C::kEStage + j * kEBytes), 128));
-#pragma unroll
-              for (int k = 0; k < kBK / 64; ++k) {
-                mma_sp_f8f6f4(d, sw64_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 64 * k),
-                              te + 2 * k, C::kIdesc, k > 0 ? 1u : 0u);
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < kBK / 32; ++k) {
-                mma_f8f6f4(d, sw128_kmajor_desc(a0 + 32 * k), sw128_kmajor_desc(b0 + 32 * k),
-                           C::kIdesc, k > 0 ? 1u : 0u);
-              }
-            }
-            mma_commit(&tfull[tb]);
-            if (++tb == C::kBufs) {
-              tb = 0;
-              tphase ^= 1u;
+          } else {
+            if (elect_one()) {
+              mma_f8f6f4_c<false>(d, da, db, C::kIdesc);
+              mma_f8f6f4_c<true>(d, da + (32 >> 4), db + (32 >> 4), C::kIdesc);
+              mma_f8f6f4_c<true>(d, da + (64 >> 4), db + (64 >> 4), C::kIdesc);
+              mma_f8f6f4_c<true>(d, da + (96 >> 4), db + (96 >> 4), C::kIdesc);
+              mma_commit(&tfull[tb]);
             }
           }
-          // the stage is free once every MMA that reads it has completed
-          mma_commit(&empty[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          __syncwarp();
+          if (++tb == C::kBufs) {
+            tb = 0;
+            tphase ^= 1u;
           }
         }
+        // the stage is free once every MMA that reads it has completed
+        if (elect_one()) mma_commit(&empty[stage]);
+        __syncwarp();
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-      if (!ok) {
-        record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
-        *abort_flag = 1;
-      }
-      // All MMAs issued must be complete before TMEM is freed.
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, kDefaultWaitCycles);
     }
+    if (!ok) {
+      record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+      *abort_flag = 1;
+    }
+    // All MMAs issued must be complete before TMEM is freed.
+    if (elect_one()) mma_commit(mma_done);
+    __syncwarp();
+    mbar_wait(mma_done, 0, kDefaultWaitCycles);
    }
   } else {
     if constexpr (kRegSplit) setmaxnreg_inc<232>();

@@ -411,6 +411,48 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 
+// The two halves of a cluster barrier. A relaxed arrive publishes nothing
+// (it follows mbarrier initialisation, which fence_mbarrier_init already
+// releases to the cluster); each thread waits exactly once per arrive.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// 16-byte store from registers into the shared memory of a CTA of the
+// cluster (`addr` from map_cluster) that counts as 16 transaction bytes on
+// that CTA's mbarrier (`bar`, also a cluster address) once it has landed.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
+                                            uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr),
+      "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)),
+      "r"(__float_as_uint(d)), "r"(bar)
+      : "memory");
+}
+
+// mbar_wait with cluster-scope acquire: for data that other CTAs of the
+// cluster stored with st_async_v4.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
 // Address of the same shared-memory location in cluster CTA `rank`.
 __device__ __forceinline__ uint32_t map_cluster(uint32_t local_addr, uint32_t rank) {
   uint32_t r;

@@ -54,12 +54,9 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
   if (tiles > 0x7FFFFFFF) return FP8BS_ERR_SHAPE;
   const int grid_y = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  alignas(64) CUtensorMap ty;
   if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, 128, 1, kSwizzle128B)) return st;
   if (int st = encode_tmap_kblocks(&tb, qw, 128, N, KB, K, BN, 1, kSwizzle128B)) return st;
-  // Y for the TMA stores of the epilogue: boxes of 128 rows x 64 bf16
-  if (int st = encode_tmap_2d(&ty, y, 2, N, M, N * 2, 64, 128, kSwizzle128B)) return st;
-  return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ty, a, grid_y, 1, stream);
+  return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
 }
 
 }  // namespace fp8bs

@@ -64,6 +64,17 @@ struct GemmArgs {
   int* err;             // device error word
 };
 
+// Split-K over a cluster of S CTAs: rank q reduces weight rows
+// [recv_lo(q, S), recv_lo(q + 1, S)) of the 128-row tile (multiples of 4).
+__host__ __device__ constexpr int recv_lo(int q, int S) { return 4 * (32 * q / S); }
+__host__ __device__ constexpr int recv_rows(int q, int S) { return recv_lo(q + 1, S) - recv_lo(q, S); }
+__host__ __device__ constexpr int recv_rows_max(int S) { return 4 * ((32 + S - 1) / S); }
+static_assert(8 * recv_rows_max(8) <= 144 && 7 * recv_rows_max(7) <= 144 &&
+                  6 * recv_rows_max(6) <= 144 && 5 * recv_rows_max(5) <= 144 &&
+                  4 * recv_rows_max(4) <= 144 && 3 * recv_rows_max(3) <= 144 &&
+                  2 * recv_rows_max(2) <= 144,
+              "receive buffer: S slots of recv_rows_max(S) rows fit 144 rows");
+
 template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
 struct Cfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
@@ -113,7 +124,22 @@ struct Cfg {
   // of 128 rows x 64 columns (128 bytes, 128-byte swizzle), 16 KB each
   static constexpr int kOffOut = (kOffTab + kTabBytes + 1023) / 1024 * 1024;
   static constexpr int kOutBytes = kSwap ? 0 : 128 * BN * 2;
-  static constexpr int kSmemBytes = kOffOut + kOutBytes + 1024;  // + slack to align the base
+  // decode order, one region used two ways: without a K split, the staging
+  // buffers of the output TMA stores (per epilogue warpgroup, kChunk tokens x
+  // 128 weight rows of bf16, token-major); with a K split, when it fits next
+  // to the stages, the receive buffer of the push reduction (one slot of
+  // recv_rows_max(S) weight rows x BN fp32 per CTA of the cluster, at most
+  // 144 rows for S <= 8) and its mbarrier
+  static constexpr int kChunk = kCols < 32 ? kCols : 32;
+  static constexpr int kYstBytes = kSwap ? kEpiWG * kChunk * 256 : 0;
+  static constexpr int kOffRecv = kOffOut + kOutBytes;
+  static constexpr int kRecvBytes = 144 * BN * 4;
+  static constexpr bool kPush =
+      kSwap && kOffRecv + (kRecvBytes > kYstBytes ? kRecvBytes : kYstBytes) + 8 + 1024 <= 227 * 1024;
+  static constexpr int kRegionBytes = kPush && kRecvBytes > kYstBytes ? kRecvBytes : kYstBytes;
+  static constexpr int kOffRecvBar = kOffRecv + kRegionBytes;
+  static constexpr int kSmemBytes =
+      kOffRecvBar + (kPush ? 8 : 0) + 1024;  // + slack to align the base
   // split-K partial tile [BN][128] fp32 reuses the (drained) stage buffers
   static_assert(BN * 128 * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -140,8 +166,10 @@ template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
 __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>::kThreads, 1)
     block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
-                      const __grid_constant__ CUtensorMap tmap_e, const GemmArgs args) {
-  // tmap_e: the 2:4 metadata (sparse) or the output Y (prefill order)
+                      const __grid_constant__ CUtensorMap tmap_e,
+                      const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
+  // tmap_e: the 2:4 metadata (sparse only); tmap_y: the output Y for the TMA
+  // stores of the epilogue
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -155,6 +183,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   uint64_t* tempty = tfull + C::kBufs;
   uint64_t* mma_done = tempty + C::kBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
+  uint64_t* recv_bar = reinterpret_cast<uint64_t*>(smem + C::kOffRecvBar);   // kPush only
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
 
   const int warp = threadIdx.x >> 5;
@@ -181,8 +210,18 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
       mbar_init(&tempty[i], 4 * kEpiWG);
     }
     mbar_init(mma_done, 1);
+    if (C::kPush && args.splits > 1) {
+      mbar_init(recv_bar, 1);
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
+    if (C::kPush && args.splits > 1) {
+      // phase 0 completes when every CTA of the cluster (this one included)
+      // has stored this CTA's rows of its partial tile
+      const int S = args.splits, rank = static_cast<int>(cluster_ctarank());
+      const int rows = recv_rows(rank, S);
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(S * rows * BN * 4));
+    }
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
     if constexpr (kSparse) tma_prefetch_desc(&tmap_e);
@@ -194,6 +233,9 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the receive barriers of the cluster are initialised before any CTA
+  // stores into them (the matching wait precedes the stores)
+  if (C::kPush && args.splits > 1) cluster_arrive_relaxed();
   const uint32_t tmem_base = *tmem_slot;
   // Dense decode order: the weight stages of the first tile are prefetched
   // into L2 while the previous kernel of the stream may still run (an L2
@@ -543,26 +585,40 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
         if (leader && ok) {
 #pragma unroll
           for (int b = 0; b < C::kCols / 64; ++b)
-            tma_store_2d(&tmap_e, out + b * 16384, ct * BN + col0 + b * 64, rt * 128);
+            tma_store_2d(&tmap_y, out + b * 16384, ct * BN + col0 + b * 64, rt * 128);
           bulk_commit_group();
         }
-      } else if (ok && args.splits == 1) {
-        // column j of the tile is token ct*BN + col0 + j; row is weight row n
-        const int n = rt * 128 + row;
-        if (n < args.N) {
+      } else if (args.splits == 1) {
+        // Column j of the tile is token ct*BN + col0 + j, the lane's row is
+        // weight row rt*128 + row: the tile goes out transposed. Per chunk of
+        // kChunk tokens, every thread writes its row's bf16 values into the
+        // token-major staging buffer (256 bytes per token, a warp's 32 rows
+        // are 64 contiguous bytes), and the leader issues one TMA store,
+        // which clips tokens >= M and rows >= N; it runs on while the next
+        // chunk or tile is computed.
+        const bool leader = (warp & 3) == 0 && lane == 0;
+        uint8_t* stage_y = smem + C::kOffRecv + wg * C::kChunk * 256;
 #pragma unroll
-          for (int j = 0; j < C::kCols; ++j) {
-            const int tok = ct * BN + col0 + j;
-            if (tok < args.M)
-              args.y[static_cast<int64_t>(tok) * args.N + n] = __float2bfloat16_rn(acc[j]);
+        for (int c = 0; c < C::kCols; c += C::kChunk) {
+          if (leader) bulk_wait_group_read0();
+          named_bar_sync(2 + wg, 128);
+          if (ok) {
+#pragma unroll
+            for (int j = 0; j < C::kChunk; ++j)
+              *reinterpret_cast<__nv_bfloat16*>(stage_y + j * 256 + row * 2) =
+                  __float2bfloat16_rn(acc[c + j]);
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2 + wg, 128);
+          if (leader && ok) {
+            tma_store_2d(&tmap_y, stage_y, rt * 128, ct * BN + col0 + c);
+            bulk_commit_group();
           }
         }
       }
     }
-    // prefill: the last stores have finished before the CTA exits
-    if constexpr (!kSwap) {
-      if ((warp & 3) == 0 && lane == 0) bulk_wait_group0();
-    }
+    // the last TMA stores have finished before the CTA exits
+    if ((warp & 3) == 0 && lane == 0) bulk_wait_group0();
     if (!ok) {
       record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
       *abort_flag = 1;
@@ -572,7 +628,78 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   tc_fence_before();
   __syncthreads();
 
-  if (kSwap && args.splits > 1) {
+  if (C::kPush && args.splits > 1) {
+    // ------------------------------- split-K reduction in the cluster, pushed --
+    // Rank q of the cluster owns weight rows [recv_lo(q), recv_lo(q + 1)) of
+    // the tile. Every epilogue thread stores its row of the fp32 partial tile
+    // straight from registers into slot `rank` of the owner's receive buffer
+    // (st.async, counted on the owner's receive barrier); each CTA then sums
+    // its slots over ranks 0..S-1 in that order and writes its rows of Y.
+    // No cluster-wide release barrier is needed: the receive barrier's
+    // transaction count says when the data is there, and a CTA never reads
+    // another CTA's memory.
+    const int S = args.splits;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int slot_rows = recv_rows_max(S);
+    float* recv = reinterpret_cast<float*>(smem + C::kOffRecv);
+    cluster_wait();
+    if (warp >= 4) {
+      const int wg = (warp - 4) >> 2;
+      const int row = (warp & 3) * 32 + lane;
+      int q = 0;
+      while (q + 1 < S && row >= recv_lo(q + 1, S)) ++q;
+      const uint32_t dst = map_cluster(
+          smem_u32(recv + (rank * slot_rows + row - recv_lo(q, S)) * BN + wg * C::kCols),
+          static_cast<uint32_t>(q));
+      const uint32_t bar = map_cluster(smem_u32(recv_bar), static_cast<uint32_t>(q));
+#pragma unroll
+      for (int j = 0; j < C::kCols; j += 4)
+        st_async_v4(dst + 4 * j, acc[j], acc[j + 1], acc[j + 2], acc[j + 3], bar);
+    }
+    bool got = mbar_wait_cluster(recv_bar, 0, limit);
+    if (!got) {
+      record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
+      // stores still in flight must land before this CTA's memory goes away
+      mbar_wait_cluster(recv_bar, 0, kDefaultWaitCycles);
+    }
+    if (got && !*abort_flag) {
+      int last_rt, last_ct;  // split-K CTAs own exactly one tile: blockIdx.y
+      tile_coords(blockIdx.y, args.row_tiles, args.col_tiles, last_rt, last_ct);
+      const int r_lo = recv_lo(rank, S);
+      const int nr4 = recv_rows(rank, S) / 4;
+      const int tok_left = args.M - last_ct * BN;
+      const int n_tok = tok_left < BN ? tok_left : BN;
+      // token index fastest: the threads of a warp read consecutive words
+      for (int idx = threadIdx.x; idx < n_tok * nr4; idx += C::kThreads) {
+        const int r4 = (idx / n_tok) * 4;
+        const int j = idx - (idx / n_tok) * n_tok;
+        float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < S) {
+            const float* p = recv + (q * slot_rows + r4) * BN + j;
+            if (q == 0) {
+              acc4 = make_float4(p[0], p[BN], p[2 * BN], p[3 * BN]);
+            } else {
+              acc4.x += p[0];
+              acc4.y += p[BN];
+              acc4.z += p[2 * BN];
+              acc4.w += p[3 * BN];
+            }
+          }
+        }
+        const int out_row = last_ct * BN + j;            // token
+        const int out_col = last_rt * 128 + r_lo + r4;   // weight row
+        if (out_col < args.N) {
+          uint2 pk;
+          pk.x = pack_bf16x2(acc4.x, acc4.y);
+          pk.y = pack_bf16x2(acc4.z, acc4.w);
+          *reinterpret_cast<uint2*>(args.y + static_cast<int64_t>(out_row) * args.N + out_col) =
+              pk;
+        }
+      }
+    }
+  } else if (kSwap && args.splits > 1) {
     // ---------------------------------------- split-K reduction in the cluster --
     // Each CTA publishes its fp32 partial tile [BN][128] (token-major, MMA row
     // index contiguous) in its own drained stage memory; rank r then sums, over
@@ -675,6 +802,15 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
                const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
   // (grid_y, splits) as chosen by the shape heuristic; adjusted below.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
+  // Y [M][N] bf16 for the epilogue's TMA stores: prefill boxes of 128 token
+  // rows x 64 columns (128-byte swizzle), decode boxes of kChunk tokens x 128
+  // weight rows (plain)
+  alignas(64) CUtensorMap ty;
+  if (int st = kSwap ? encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2, 128,
+                                      C::kChunk, kSwizzleNone)
+                     : encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2, 64,
+                                      128, kSwizzle128B))
+    return st;
   auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   static std::once_flag flags[64];
   int dev = 0;
@@ -719,7 +855,7 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
     attrs[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, te, args) != cudaSuccess) return FP8BS_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, args) != cudaSuccess) return FP8BS_ERR_CUDA;
   return FP8BS_OK;
 }
 

@@ -215,11 +215,15 @@ def test_output_guard_bands_untouched():
     assert not torch.isnan(y).any()
 
 
-def test_bounded_wait_reports_timeout_and_recovers():
+@pytest.mark.parametrize("M", [8, 64])
+def test_bounded_wait_reports_timeout_and_recovers(M):
     """A wait limit of one cycle makes the kernel give up its first wait that
     is not already satisfied: it records FP8BS_ERR_DEVICE_TIMEOUT, drains its
-    own copies and MMAs, and the next call with the default limit is correct."""
-    M, N, K = 64, 4096, 4096
+    own copies and MMAs, and the next call with the default limit is correct.
+    Both shapes split K over a cluster of 4 CTAs: M = 8 reduces by pushing
+    partial rows into the owner CTA's receive buffer, M = 64 by reading the
+    other CTAs' shared memory."""
+    N, K = 4096, 4096
     qa, sa, qw, sw = _quantized("llama", M, N, K, 11)
     args = [to_dev(a) for a in (qa, sa, qw, sw)]
     fb.get_device_error()

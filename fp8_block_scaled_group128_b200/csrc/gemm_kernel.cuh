@@ -411,13 +411,16 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     // block). The groups of this CTA are (tile, kbg) for its tiles in order and
     // kbg = kb0, kb0 + kG, ... < kb1.
     int g_tile = blockIdx.y, g_kb = kb0;   // next group to stage
+    // coordinates of g_tile, recomputed only when it changes (the grouped
+    // raster costs three integer divisions, a long dependency chain that
+    // would otherwise stall every group boundary)
+    int grt = 0, gct = 0;
+    if (g_tile < num_tiles) tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
     // raw loads of the next group; multiplied only when stored, a group
     // later, so that nothing waits on them
     float pre_a[C::kPer], pre_w[C::kPer];
     auto group_load = [&]() {
       if (g_tile >= num_tiles) return;
-      int grt, gct;
-      tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
 #pragma unroll
       for (int i = 0; i < C::kPer; ++i) {
         const int idx = e + C::kEpiThreads * i;
@@ -456,6 +459,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
       if (g_kb >= kb1) {
         g_kb = kb0;
         g_tile += gridDim.y;
+        if (g_tile < num_tiles) tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
       }
     };
     group_load();

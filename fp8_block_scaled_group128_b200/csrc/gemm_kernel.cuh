@@ -415,32 +415,51 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     // raster costs three integer divisions, a long dependency chain that
     // would otherwise stall every group boundary)
     int grt = 0, gct = 0;
-    if (g_tile < num_tiles) tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
+    // Thread e stages table entries (K-block sg of the group, slot s0 + i *
+    // kSlotStep) for i < kPer: the same K-block for every i. In decode order
+    // its first token and the scale pointers at K-block sg are fixed per
+    // tile, so a group boundary only adds the group's first K-block to them
+    // (prefill, short of registers, recomputes them per group).
+    constexpr int kSlotStep = C::kEpiThreads / kG;
+    static_assert(C::kEpiThreads % kG == 0 && (kSwap || 128 % kSlotStep == 0), "table slots");
+    const int sg = e % kG, s0 = e / kG;
+    int first = 0, nb0 = 0;                 // first token (decode) or row (prefill); weight block
+    const float* a0 = args.sa;
+    const float* w0 = args.sw;
+    auto tile_bases = [&]() {
+      tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
+      if constexpr (kSwap) {
+        first = gct * BN + s0;
+        nb0 = grt;
+        a0 = args.sa + static_cast<int64_t>(first) * KB + sg;
+        w0 = args.sw + static_cast<int64_t>(nb0) * KB + sg;
+      }
+    };
+    if (g_tile < num_tiles) tile_bases();
     // raw loads of the next group; multiplied only when stored, a group
     // later, so that nothing waits on them
     float pre_a[C::kPer], pre_w[C::kPer];
     auto group_load = [&]() {
       if (g_tile >= num_tiles) return;
+      const bool kb_ok = g_kb + sg < kb1;
 #pragma unroll
       for (int i = 0; i < C::kPer; ++i) {
-        const int idx = e + C::kEpiThreads * i;
-        const int g = idx % kG, slot = idx / kG;
-        const int kb = g_kb + g;
+        const int d = i * kSlotStep;   // slot offset from s0
         float va = 0.0f, vw = 0.0f;
-        if (kb < kb1) {
-          if constexpr (kSwap) {
-            const int64_t tok = static_cast<int64_t>(gct) * BN + slot;
-            if (tok < args.M) {
-              va = args.sa[tok * KB + kb];
-              vw = args.sw[grt * KB + kb];
-            }
-          } else {
-            const int64_t m = static_cast<int64_t>(grt) * 128 + (slot & 127);
-            const int nb = (gct * BN + (slot >> 7) * C::kCols) / 128;
-            if (m < args.M && nb < args.NB) {
-              va = args.sa[m * KB + kb];
-              vw = args.sw[nb * KB + kb];
-            }
+        if constexpr (kSwap) {
+          if (kb_ok && first + d < args.M) {
+            va = a0[static_cast<int64_t>(d) * KB + g_kb];
+            vw = w0[g_kb];
+          }
+        } else {
+          // slot s0 + d is token row s0 + (d & 127) of the tile, weight block
+          // gct * BN / 128 + (d >> 7) * kCols / 128
+          const int64_t m = static_cast<int64_t>(grt) * 128 + s0 + (d & 127);
+          const int nb = (gct * BN + (d >> 7) * C::kCols) / 128;
+          const int kb = g_kb + sg;
+          if (kb_ok && m < args.M && nb < args.NB) {
+            va = args.sa[m * KB + kb];
+            vw = args.sw[nb * KB + kb];
           }
         }
         pre_a[i] = va;
@@ -449,17 +468,15 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     };
     auto group_store = [&](int buf) {
 #pragma unroll
-      for (int i = 0; i < C::kPer; ++i) {
-        const int idx = e + C::kEpiThreads * i;
-        tab[(buf * kG + idx % kG) * C::kTabStride + idx / kG] = pre_a[i] * pre_w[i];
-      }
+      for (int i = 0; i < C::kPer; ++i)
+        tab[(buf * kG + sg) * C::kTabStride + s0 + i * kSlotStep] = pre_a[i] * pre_w[i];
     };
     auto group_next = [&]() {
       g_kb += kG;
       if (g_kb >= kb1) {
         g_kb = kb0;
         g_tile += gridDim.y;
-        if (g_tile < num_tiles) tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
+        if (g_tile < num_tiles) tile_bases();
       }
     };
     group_load();

@@ -93,12 +93,17 @@ struct Cfg {
   static constexpr int kThreads = 128 * (1 + kEpiWG);
   static constexpr int kCols = BN / kEpiWG;  // accumulator columns per epilogue thread
   static_assert(kCols % 16 == 0 && kCols <= 128, "epilogue column split");
+  // Decode order: two warps issue the MMAs, alternating K-blocks (the
+  // issue of a K-block's tcgen05 operations, ~300 cycles, paces the small
+  // tiles otherwise).
+  static constexpr bool kDualIssue = kSwap;
   // TMEM: kBufs partial buffers of BN columns (up to 8, so the MMA can run
   // ahead of the promotion), then (sparse) two metadata buffers of 4
-  // columns; the allocation is a power of two >= 32.
-  static constexpr int kBufs = (512 - (kSparse ? 8 : 0)) / BN < 8 ? (512 - (kSparse ? 8 : 0)) / BN : 8;
+  // columns per issuing warp; the allocation is a power of two >= 32.
+  static constexpr int kMetaCols = kSparse ? 8 * (kDualIssue ? 2 : 1) : 0;
+  static constexpr int kBufs = (512 - kMetaCols) / BN < 8 ? (512 - kMetaCols) / BN : 8;
   static_assert(kBufs >= 2, "at least two TMEM partial buffers");
-  static constexpr int kTmemUsed = kBufs * BN + (kSparse ? 8 : 0);
+  static constexpr int kTmemUsed = kBufs * BN + kMetaCols;
   static constexpr int kTmemCols =
       kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128 : kTmemUsed <= 256 ? 256 : 512;
   static_assert(kTmemUsed <= 512, "TMEM has 512 columns");
@@ -203,13 +208,13 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], C::kDualIssue ? 2 : 1);
     }
     for (int i = 0; i < C::kBufs; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 4 * kEpiWG);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, C::kDualIssue ? 2 : 1);
     if (C::kPush && args.splits > 1) {
       mbar_init(recv_bar, 1);
     }
@@ -309,15 +314,20 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
       }
       mbar_wait(&full[s], ph, kDefaultWaitCycles);
     }
-   } else if (warp == 1) {
+   } else if (warp == 1 || (C::kDualIssue && warp == 2)) {
     // ---------------------------------------------------------- MMA issuer --
     // The whole warp runs the loop (warp-uniform operands); one elected lane
-    // issues each tcgen05 operation.
+    // issues each tcgen05 operation. With two issuing warps, warp 1 + i
+    // issues the K-blocks whose running index has parity i; both walk the
+    // whole sequence (stages, partial buffers and their phases) and both
+    // release each stage and the final barrier.
+    const uint32_t me = static_cast<uint32_t>(warp - 1);
     int stage = 0;
     uint32_t phase = 0;
     int tb = 0;
     uint32_t tphase = 0;
-    uint32_t e_buf = 0;  // sparse: TMEM metadata buffer, alternating per K-block
+    uint32_t kcount = 0;  // running K-block index of this CTA
+    uint32_t e_buf = 0;   // sparse: this warp's TMEM metadata buffer, alternating
     bool ok = true;
     // Shared-memory descriptors of stage 0, K-block 0; every other operand
     // tile is an offset from them: the start-address field is address >> 4 in
@@ -336,6 +346,15 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
 #pragma unroll
         for (int j = 0; j < kKS; ++j) {
           if (kb + j >= kb1) break;
+          const bool mine = !C::kDualIssue || (kcount & 1u) == me;
+          ++kcount;
+          if (!mine) {
+            if (++tb == C::kBufs) {
+              tb = 0;
+              tphase ^= 1u;
+            }
+            continue;
+          }
           if (!mbar_wait(&tempty[tb], tphase ^ 1u, limit)) {
             ok = false;
             break;
@@ -348,7 +367,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
             // metadata of this K-block -> TMEM (4 columns, lane = weight
             // row), then two sparse MMAs of logical depth 64 (32 compressed
             // bytes of A and 64 bytes of B each), reading 2 metadata columns
-            const uint32_t te = tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 4u * e_buf;
+            const uint32_t te =
+                tmem_base + static_cast<uint32_t>(C::kBufs * BN) + 8u * me + 4u * e_buf;
             e_buf ^= 1u;
             const uint64_t de = de0 + static_cast<uint32_t>((stage * C::kEStage + j * kEBytes) >> 4);
             if (elect_one()) {

@@ -180,6 +180,12 @@ __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Prefetch the global-memory line holding `p` into L2 (no completion; it
+// never changes what a later load reads).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 // Prefetch a 3-D box of a tensor into L2 (no shared memory, no completion;
 // it never changes what a later load reads).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t x, int32_t y,

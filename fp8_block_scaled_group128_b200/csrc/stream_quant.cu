@@ -289,11 +289,22 @@ template <int kGroups>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const __nv_bfloat16* __restrict__ x, int64_t groups,
                      uint8_t* __restrict__ q, float* __restrict__ scale) {
-  grid_dependency_wait();
-  grid_launch_dependents();
   const int64_t teams = static_cast<int64_t>(gridDim.x) * (kActThreads / 16);
   const int64_t team = static_cast<int64_t>(blockIdx.x) * (kActThreads / 16) + (threadIdx.x >> 4);
   const int chunk = threadIdx.x & 15;
+  // While the previous kernel of the stream may still run, bring this
+  // thread's input lines into L2 (one thread per 128-byte line): the
+  // prefetch never changes what the loads below read, even if that kernel
+  // writes x, and when it does not, the HBM latency overlaps the wait.
+  if ((chunk & 7) == 0) {
+#pragma unroll
+    for (int j = 0; j < kGroups; ++j) {
+      const int64_t g = team + j * teams;
+      if (g < groups) prefetch_l2(reinterpret_cast<const uint4*>(x + g * 128) + chunk);
+    }
+  }
+  grid_dependency_wait();
+  grid_launch_dependents();
   uint4 v[kGroups];
 #pragma unroll
   for (int j = 0; j < kGroups; ++j) {

@@ -149,7 +149,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
   }
   __syncthreads();
   // No global memory was touched so far; the input may come from the
-  // previous kernel of the stream.
+  // previous kernel of the stream. Its first tiles are prefetched into L2
+  // meanwhile (a prefetch never changes what a later load reads).
+  if (t == 0) {
+    Cursor pf = load;
+    for (int s = 0; s < kQStages; ++s) {
+      if (first + s * step >= a.num_tiles) break;
+      tma_prefetch_l2_2d(&tmap_x, pf.kb * 128, pf.rb * 128);
+      advance(pf);
+    }
+  }
   grid_dependency_wait();
   grid_launch_dependents();
   int issued = 0;

@@ -242,17 +242,21 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   // stores into them (the matching wait precedes the stores)
   if (C::kPush && args.splits > 1) cluster_arrive_relaxed();
   const uint32_t tmem_base = *tmem_slot;
-  // Dense decode order: the weight stages of the first tile are prefetched
-  // into L2 while the previous kernel of the stream may still run (an L2
-  // prefetch never changes what a later load reads, so this is safe even if
-  // that kernel writes the weights). Measured: 3-7 % faster dense decode
-  // launches; the 2:4 launches ran slower with it, so they do without.
-  if constexpr (kSwap && !kSparse) {
+  // Decode order: the weight stages of the first tile (values and metadata
+  // for 2:4) are prefetched into L2 while the previous kernel of the stream
+  // may still run (an L2 prefetch never changes what a later load reads, so
+  // this is safe even if that kernel writes the weights). Measured: 3-7 %
+  // faster dense launches; 2:4 launches gain at 32 tokens and more (M = 128
+  // four-linear sequence 75.3 -> 72.6 us, 2:4 prefill +4 %) and lose up to
+  // 1 us at 16, so those do without.
+  if constexpr (kSwap && (!kSparse || BN >= 32)) {
     if (threadIdx.x == 0 && static_cast<int>(blockIdx.y) < num_tiles) {
       int rt, ct;
       tile_coords(blockIdx.y, args.row_tiles, args.col_tiles, rt, ct);
-      for (int kb = kb0, n = 0; kb < kb1 && n < kStages; kb += kKS, ++n)
+      for (int kb = kb0, n = 0; kb < kb1 && n < kStages; kb += kKS, ++n) {
         tma_prefetch_l2_3d(&tmap_a, 0, rt * 128, kb);
+        if constexpr (kSparse) tma_prefetch_l2_3d(&tmap_e, 0, rt * 128, kb);
+      }
     }
   }
   // Everything else waits: inputs may come from the previous kernel.

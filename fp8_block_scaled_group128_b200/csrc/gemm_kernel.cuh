@@ -9,17 +9,22 @@
 // is one "partial" MMA chain written fresh into TMEM, and the epilogue warps
 // promote it into fp32 register accumulators multiplied by sA * sW:
 //
-//   warp 0 (one lane)  TMA producer: K-block tiles -> shared memory, a
+//   warp 0             TMA producer: K-block tiles -> shared memory, a
 //                      kStages-deep ring of mbarriers.
-//   warp 1 (one lane)  MMA issuer: per K-block, 4 x tcgen05.mma kind::f8f6f4
+//   warp 1 (and 2)     MMA issuer: per K-block, 4 x tcgen05.mma kind::f8f6f4
 //                      (K = 32 each), or for 2:4 weights one tcgen05.cp of the
 //                      metadata into TMEM and 2 x tcgen05.mma.sp (logical K =
-//                      64 each), into TMEM partial buffer (kb % 2); commits
-//                      free the smem stage and signal the partial.
+//                      64 each), into one of kBufs TMEM partial buffers;
+//                      commits free the smem stage and signal the partial. In
+//                      decode order warps 1 and 2 issue alternate K-blocks.
+//                      Both roles run their loops warp-wide and issue from one
+//                      elected lane.
 //   warps 4..          promotion / epilogue: tcgen05.ld the partial, FMA into
-//                      registers with the K-block's scale product, hand the
-//                      TMEM buffer back; at the end of a tile, round to bf16
-//                      and store (or reduce split-K partials over the cluster).
+//                      registers with the K-block's scale product (staged per
+//                      group of kG K-blocks in a shared table), hand the TMEM
+//                      buffer back; at the end of a tile, round to bf16 and
+//                      store through shared memory with TMA (or reduce split-K
+//                      partials over the cluster).
 //
 // Operand orders:
 //   kSwap = false (prefill, dense): MMA rows = tokens (128), MMA cols =
@@ -28,7 +33,9 @@
 //     MMA cols = tokens (BN = 16..256). When the weight tiles alone do not
 //     fill the GPU, K is split over a thread-block cluster of `splits` CTAs
 //     that sum their partial tiles through distributed shared memory in rank
-//     order, so results are deterministic and no global scratch is used.
+//     order (pushed into the owner's receive buffer, or pulled from the other
+//     CTAs' stage memory), so results are deterministic and no global scratch
+//     is used.
 // Without a K split the CTAs are persistent: CTA y walks tiles y, y+gridDim.y...
 //
 // Every mbarrier wait is bounded; a wait that runs out records

@@ -564,7 +564,7 @@ def run_ours(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 -> fp32 accumulate, bf16 out",
-        "data": "synthetic (seeded bf16, Llama-3-8B linear shapes; see DESIGN.md)",
+        "data": "synthetic (seeded bf16, Llama-3-8B linear shapes)",
         "config": {"workload": WORKLOAD, "rows": list(ROWS), "linears_NK": [list(l) for l in LINEARS],
                    "tokens_M": list(TOKENS), "global_batch": sum(TOKENS) * world,
                    "step_bytes": sb, "launches_per_step": per_step_launches,

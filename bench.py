@@ -312,8 +312,11 @@ def fp8_tensor_peak():
 
 def run_prefill(dev, stream, world, reps=10):
     """Prefill-shaped GEMMs timed on their own: the dense GEMM at M in {2048,
-    8192} on the four Llama-3-8B linears and the LM head, and the 2:4 GEMM at
-    M = 4096 on its two shapes. Each shape's launches are replayed from a CUDA
+    8192} on the four Llama-3-8B linears and the LM head, the 2:4 GEMM at
+    M = 4096 on its two shapes, and on the down projection at M = 8192 the GEMM
+    with the next layer's 1x128 quantization fused into its epilogue
+    ("fused", codes only) against the GEMM followed by the activation
+    quantizer ("separate"). Each shape's launches are replayed from a CUDA
     graph of `reps` back-to-back launches (one warm-up replay, three timed),
     CUDA events on the launching stream. Inputs: the seeded synthetic llama
     tensors, quantized / compressed on the device before timing."""
@@ -323,23 +326,34 @@ def run_prefill(dev, stream, world, reps=10):
     shapes = [("dense", M, N, K) for M in synth.PREFILL_M
               for N, K in synth.LLAMA3_8B_LINEARS + (synth.LLAMA3_8B_LM_HEAD,)]
     shapes += [("sparse", 4096, N, K) for N, K in synth.SPARSE_LINEARS]
+    shapes += [(kind, 8192, 4096, 14336) for kind in ("fused", "separate")]
     rows, tot_flop, tot_ms = [], 0.0, 0.0
     wcache = {}
     for kind, M, N, K in shapes:
         with torch.cuda.stream(stream):
-            key = (kind, N, K)
+            key = (kind == "sparse", N, K)
             if key not in wcache:
                 wcache.clear()
                 w = synth.weights("llama", N, K, seed=7).to(dev)
-                wcache[key] = (fb.fp8_quant_weight_block128(w) if kind == "dense"
-                               else fb.prune24_compress(w)[:3])
+                wcache[key] = (fb.prune24_compress(w)[:3] if kind == "sparse"
+                               else fb.fp8_quant_weight_block128(w))
                 del w
             x = synth.activations("llama", M, K, seed=7).to(dev)
             qa, sa = fb.fp8_quant_act_group128(x)
             y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
             wq = wcache[key]
-            fn = ((lambda: fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y)) if kind == "dense" else
-                  (lambda: fb.fp8_sparse24_gemm(qa, sa, wq[0], wq[1], wq[2], y=y)))
+            qy = torch.empty(M, N, dtype=torch.uint8, device=dev)
+            sy = torch.empty(M, N // 128, dtype=torch.float32, device=dev)
+            if kind == "dense":
+                fn = lambda: fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y)  # noqa: E731
+            elif kind == "sparse":
+                fn = lambda: fb.fp8_sparse24_gemm(qa, sa, wq[0], wq[1], wq[2], y=y)  # noqa: E731
+            elif kind == "fused":
+                fn = lambda: fb.fp8_block_gemm_quant(  # noqa: E731
+                    qa, sa, wq[0], wq[1], qy=qy, sy=sy, want_y=False)
+            else:
+                fn = lambda: (fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y),  # noqa: E731
+                              fb.fp8_quant_act_group128(y, qa=qy, sa=sy))
             fn()
         stream.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -358,20 +372,22 @@ def run_prefill(dev, stream, world, reps=10):
         assert fb.get_device_error(stream) == 0
         ms = max_over_ranks(e0.elapsed_time(e1) / (3 * reps), world)
         # algorithmic FLOPs: 2MNK dense; MNK (the kept half) for 2:4
-        flop = (2.0 if kind == "dense" else 1.0) * M * N * K
+        flop = (1.0 if kind == "sparse" else 2.0) * M * N * K
         tf = flop / (ms * 1e-3) / 1e12
         rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
                      "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4)})
         if kind == "dense":
             tot_flop += flop
             tot_ms += ms
-        del g, x, qa, sa, y
+        del g, x, qa, sa, y, qy, sy
     wcache.clear()
     torch.cuda.empty_cache()
     agg = tot_flop / (tot_ms * 1e-3) / 1e12
     return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
             "dense_achieved": round(agg, 1), "dense_frac": round(agg / peak, 4),
-            "note": "dense: 2MNK FLOPs; 2:4: MNK FLOPs (nonzero work) against the dense peak",
+            "note": "dense: 2MNK FLOPs; 2:4: MNK FLOPs (nonzero work) against the dense peak; "
+                    "fused / separate: the down projection with the next layer's 1x128 "
+                    "quantization in the epilogue / after it (not in dense_achieved)",
             "shapes": rows}
 
 

@@ -28,6 +28,7 @@ SIGNATURES = {
     "fp8_quant_weight_block128": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "prune24_compress": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "fp8_block_gemm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_block_gemm_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_sparse24_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
@@ -171,6 +172,33 @@ def fp8_block_gemm(qa, sa, qw, sw, y=None, workspace=None, stream=None):
            lib().fp8_block_gemm(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(y), M, N, K,
                                 _ptr(ws), ws_bytes, _stream(stream, qa)))
     return y
+
+
+def fp8_block_gemm_quant(qa, sa, qw, sw, y=None, qy=None, sy=None, want_y=True, workspace=None,
+                         stream=None):
+    """fp8_block_gemm plus the next layer's input quantization of its bf16 output:
+    returns (y, qy, sy) with qy, sy = fp8_quant_act_group128(y). With want_y=False
+    and M > 256, y is not written (returned as None)."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    NB, KB = -(-N // 128), K // 128
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa, torch.float32, (M, KB), "sa")
+    _dev(qw, torch.uint8, (N, K), "qw")
+    _dev(sw, torch.float32, (NB, KB), "sw")
+    if y is None and (want_y or M <= 256):
+        y = _empty((M, N), torch.bfloat16, qa.device)
+    if y is not None:
+        _dev(y, torch.bfloat16, (M, N), "y")
+    qy = _empty((M, N), torch.uint8, qa.device) if qy is None else qy
+    sy = _empty((M, N // 128), torch.float32, qa.device) if sy is None else sy
+    _dev(qy, torch.uint8, (M, N), "qy")
+    _dev(sy, torch.float32, (M, N // 128), "sy")
+    ws, ws_bytes = _workspace(M, N, K, False, qa.device, workspace)
+    _check("fp8_block_gemm_quant",
+           lib().fp8_block_gemm_quant(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(y), _ptr(qy),
+                                      _ptr(sy), M, N, K, _ptr(ws), ws_bytes, _stream(stream, qa)))
+    return y, qy, sy
 
 
 def fp8_sparse24_gemm(qa, sa, vals, meta, sw, y=None, workspace=None, stream=None):

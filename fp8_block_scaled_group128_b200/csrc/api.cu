@@ -202,6 +202,25 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
                            static_cast<cudaStream_t>(stream));
 }
 
+int fp8_block_gemm_quant(const void* qa, const float* sa, const void* qw, const float* sw,
+                         void* y_bf16, void* qy_e4m3, float* sy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (int st = check_gemm_args(M, N, K)) return st;
+  if (N % 128 != 0) return FP8BS_ERR_SHAPE;  // whole 1x128 groups of Y
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa || !qw || !sw || !qy_e4m3 || !sy) return FP8BS_ERR_NULL;
+  if (M <= 256 && !y_bf16) return FP8BS_ERR_NULL;  // decode-sized M quantizes the stored Y
+  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) ||
+      (y_bf16 && !aligned16(y_bf16)) || !aligned16(qy_e4m3) || !aligned16(sy))
+    return FP8BS_ERR_ALIGN;
+  if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 0)) return FP8BS_ERR_WORKSPACE;
+  (void)workspace;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_block_gemm(qa, sa, qw, sw, y_bf16, M, N, K, wait_limit(), err,
+                           static_cast<cudaStream_t>(stream), qy_e4m3, sy);
+}
+
 int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const uint8_t* meta,
                       const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
                       void* workspace, size_t workspace_bytes, void* stream) {

@@ -9,10 +9,10 @@ using namespace gemm_detail;
 
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,
                       int64_t M, int64_t N, int64_t K, long long wait_limit, int* err,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, void* qy, float* sy) {
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
-  GemmArgs a;
+  GemmArgs a{};
   a.sa = sa;
   a.sw = sw;
   a.y = static_cast<__nv_bfloat16*>(y);
@@ -22,9 +22,21 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   a.NB = static_cast<int>((N + 127) / 128);
   a.wait_limit = wait_limit;
   a.err = err;
+  a.qy = static_cast<uint8_t*>(qy);
+  a.sy = sy;
   alignas(64) CUtensorMap ta, tb;
 
   const uint64_t KB = static_cast<uint64_t>(K / 128);
+  if (M <= 256 && qy != nullptr) {
+    // Decode-sized M with the next layer's quantization: Y, then the
+    // activation quantizer on it (the decode-order tile holds a group of N
+    // across four warps, or across a cluster with a K split).
+    if (int st = launch_block_gemm(qa, sa, qw, sw, y, M, N, K, wait_limit, err, stream, nullptr,
+                                   nullptr))
+      return st;
+    return launch_quant_act_group128(y, M, N, qy, sy, stream) == cudaSuccess ? FP8BS_OK
+                                                                              : FP8BS_ERR_CUDA;
+  }
   if (M <= 256) {
     // Decode: weights on the MMA M side, tokens on the MMA N side; stages of
     // two K-blocks.
@@ -56,6 +68,7 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   const int grid_y = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
   if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, 128, 1, kSwizzle128B)) return st;
   if (int st = encode_tmap_kblocks(&tb, qw, 128, N, KB, K, BN, 1, kSwizzle128B)) return st;
+  if (qy != nullptr) return launch_cfg<BN, false, false, 3, 2, 1, true>(ta, tb, ta, a, grid_y, 1, stream);
   return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
 }
 

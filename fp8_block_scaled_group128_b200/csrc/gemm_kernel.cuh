@@ -48,6 +48,7 @@
 #include <tuple>
 
 #include "common.cuh"
+#include "e4m3_codec.cuh"
 #include "kernels.h"
 
 namespace fp8bs {
@@ -69,6 +70,8 @@ struct GemmArgs {
   int splits;           // K splits = cluster size along x
   long long wait_limit; // bound of each mbarrier wait, SM cycles
   int* err;             // device error word
+  uint8_t* qy;          // kQOut: Y quantized in 1x128 groups along N, [M][N] E4M3
+  float* sy;            // kQOut: their scales, [M][N/128]
 };
 
 // Split-K over a cluster of S CTAs: rank q reduces weight rows
@@ -174,15 +177,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false>
 __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>::kThreads, 1)
     block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_e,
                       const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   // tmap_e: the 2:4 metadata (sparse only); tmap_y: the output Y for the TMA
-  // stores of the epilogue
+  // stores of the epilogue. kQOut (prefill order only): the epilogue also
+  // quantizes Y for the next layer (args.qy, args.sy) and Y itself is written
+  // only if args.y is set.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
+  static_assert(!kQOut || (!kSwap && C::kCols == 128), "fused quantization: one group per thread");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -634,11 +640,37 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
         }
         fence_proxy_async_smem();
         named_bar_sync(2 + wg, 128);
-        if (leader && ok) {
+        if (leader && ok && (!kQOut || args.y != nullptr)) {
 #pragma unroll
           for (int b = 0; b < C::kCols / 64; ++b)
             tma_store_2d(&tmap_y, out + b * 16384, ct * BN + col0 + b * 64, rt * 128);
           bulk_commit_group();
+        }
+        if constexpr (kQOut) {
+          // The next layer's activation quantization, with the arithmetic of
+          // the activation quantizer on the bf16 values just stored: this
+          // thread's 128 columns of token row m are one 1x128 group of Y
+          // along N (N is a multiple of 128).
+          const int64_t m = static_cast<int64_t>(rt) * 128 + row;
+          const int n0 = ct * BN + col0;
+          if (ok && m < args.M && n0 < args.N) {
+            auto chunk8 = [&](int c) {
+              return make_uint4(pack_bf16x2(acc[c + 0], acc[c + 1]),
+                                pack_bf16x2(acc[c + 2], acc[c + 3]),
+                                pack_bf16x2(acc[c + 4], acc[c + 5]),
+                                pack_bf16x2(acc[c + 6], acc[c + 7]));
+            };
+            uint32_t mx = absmax8(chunk8(0));
+#pragma unroll
+            for (int c = 8; c < C::kCols; c += 8) mx = bf16x2_absmax(mx, absmax8(chunk8(c)));
+            const float sc = scale_of_amax(absmax_to_float(mx));
+            const ScaleDivider d(sc);
+            uint8_t* qrow = args.qy + m * args.N + n0;
+#pragma unroll
+            for (int c = 0; c < C::kCols; c += 8)
+              *reinterpret_cast<uint2*>(qrow + c) = encode8(chunk8(c), d);
+            args.sy[m * (args.N / 128) + n0 / 128] = sc;
+          }
         }
       } else if (args.splits == 1) {
         // Column j of the tile is token ct*BN + col0 + j, the lane's row is
@@ -849,21 +881,24 @@ int max_active_clusters(Kern kern, int threads, int smem, int S, int dev) {
   return n;
 }
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
                const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
   // (grid_y, splits) as chosen by the shape heuristic; adjusted below.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   // Y [M][N] bf16 for the epilogue's TMA stores: prefill boxes of 128 token
   // rows x 64 columns (128-byte swizzle), decode boxes of kChunk tokens x 128
-  // weight rows (plain)
-  alignas(64) CUtensorMap ty;
-  if (int st = kSwap ? encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2, 128,
-                                      C::kChunk, kSwizzleNone)
-                     : encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2, 64,
-                                      128, kSwizzle128B))
-    return st;
-  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
+  // weight rows (plain). Without Y (a fused quantization that writes only the
+  // codes) the map stays zero and is never used.
+  alignas(64) CUtensorMap ty{};
+  if (a.y != nullptr) {
+    if (int st = kSwap ? encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
+                                        128, C::kChunk, kSwizzleNone)
+                       : encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
+                                        64, 128, kSwizzle128B))
+      return st;
+  }
+  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS, kQOut>;
   static std::once_flag flags[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8BS_ERR_CUDA;

@@ -20,7 +20,7 @@ int launch_sparse24_gemm(const void* qa, const float* sa, const void* vals, cons
                          long long wait_limit, int* err, cudaStream_t stream) {
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
-  GemmArgs a;
+  GemmArgs a{};
   a.sa = sa;
   a.sw = sw;
   a.y = static_cast<__nv_bfloat16*>(y);

@@ -15,10 +15,11 @@ cudaError_t launch_prune24_compress(const void* w, int64_t N, int64_t K, void* v
                                     uint8_t* meta, float* sw, void* w_pruned,
                                     cudaStream_t stream);
 
-// Dense block-scaled GEMM. Returns FP8BS_* status.
+// Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
+// N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,
                       int64_t M, int64_t N, int64_t K, long long wait_limit, int* err,
-                      cudaStream_t stream);
+                      cudaStream_t stream, void* qy = nullptr, float* sy = nullptr);
 
 // 2:4 sparse block-scaled GEMM. Returns FP8BS_* status.
 int launch_sparse24_gemm(const void* qa, const float* sa, const void* vals, const uint8_t* meta,

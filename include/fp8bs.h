@@ -126,6 +126,26 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
                    void* stream);
 
 /*
+ * fp8_block_gemm with the next layer's input quantization fused in: the same
+ * y, and qy / sy = fp8_quant_act_group128(y) of that bf16 y, i.e. y's rows
+ * cut into 1x128 groups along N ("FP8 à granularité fine": the output of one
+ * linear is the activation of the next, quantized per token per 128
+ * channels). For M > 256 the GEMM's epilogue quantizes its own tile (each
+ * promotion thread holds one group); for M <= 256 y is written and then
+ * quantized by the activation quantizer.
+ *
+ *   y_bf16  [M][N] bf16, output; may be NULL when M > 256 (then only the codes
+ *           are written), required when M <= 256.
+ *   qy_e4m3 [M][N] E4M3 codes, output; sy [M][N/128] fp32 scales, output.
+ *   N must be a multiple of 128; the other arguments as fp8_block_gemm.
+ * Returns FP8BS_ERR_SHAPE for N % 128 != 0 and FP8BS_ERR_NULL for a missing
+ * qy / sy (or y with M <= 256).
+ */
+int fp8_block_gemm_quant(const void* qa, const float* sa, const void* qw, const float* sw,
+                         void* y_bf16, void* qy_e4m3, float* sy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The block-scaled GEMM with 2:4-compressed weights (vals, meta, sw as written
  * by prune24_compress). Same result definition as fp8_block_gemm with qw the
  * decompressed codes (pruned positions are code 0).

@@ -83,3 +83,17 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.fp8_block_gemm(BAD, BAD, BAD, None, BAD, 4, 8, 128, None, 0, None) == 1
     assert lib.fp8_block_gemm(BAD, BAD, MIS, BAD, BAD, 4, 8, 128, None, 0, None) == 3
     assert lib.prune24_compress(BAD, 4, 128, BAD, BAD, BAD, MIS, None) == 3
+
+
+def test_fused_quantization_argument_checks(lib):
+    """fp8_block_gemm_quant: whole 1x128 groups of y (N % 128), the codes and
+    scales are required, and y is required when M <= 256 (that path quantizes
+    the stored y); all checked before any launch."""
+    g = lib.fp8_block_gemm_quant
+    assert g(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 4, 136, 128, None, 0, None) == 2
+    assert g(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 4, 128, 100, None, 0, None) == 2
+    assert g(BAD, BAD, BAD, BAD, BAD, None, BAD, 4, 128, 128, None, 0, None) == 1
+    assert g(BAD, BAD, BAD, BAD, BAD, BAD, None, 4, 128, 128, None, 0, None) == 1
+    assert g(BAD, BAD, BAD, BAD, None, BAD, BAD, 256, 128, 128, None, 0, None) == 1
+    assert g(BAD, BAD, BAD, BAD, BAD, MIS, BAD, 4, 128, 128, None, 0, None) == 3
+    assert g(None, None, None, None, None, None, None, 0, 128, 128, None, 0, None) == 0

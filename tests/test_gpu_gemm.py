@@ -237,3 +237,28 @@ def test_bounded_wait_reports_timeout_and_recovers(M):
     assert fb.get_device_error() == 0
     check_gemm(y, oracle.block_gemm(qa, sa, qw, sw), oracle.gemm_error_bound(qa, sa, qw, sw),
                "after timeout")
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 4096, 4096), (128, 6144, 4096), (300, 640, 512),
+                                   (2048, 6144, 4096), (4096, 2048, 1024)])
+def test_gemm_with_fused_next_layer_quantization(M, N, K):
+    """fp8_block_gemm_quant gives fp8_block_gemm's y, byte for byte, and the
+    next layer's 1x128 codes and scales of that bf16 y exactly as the oracle's
+    activation quantizer computes them; with M > 256 (the fused epilogue) also
+    when y itself is not written. N = 640 leaves the second warpgroup of the
+    last column tile without a group."""
+    qa, sa, qw, sw = _quantized("llama", M, N, K, 3)
+    args = [to_dev(a) for a in (qa, sa, qw, sw)]
+    y_plain = fb.fp8_block_gemm(*args)
+    y, qy, sy = fb.fp8_block_gemm_quant(*args)
+    torch.cuda.synchronize()
+    assert fb.get_device_error() == 0
+    assert torch.equal(y, y_plain)
+    q_ref, s_ref = oracle.quant_act_group128(y.cpu())
+    np.testing.assert_array_equal(qy.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(sy.cpu().numpy(), s_ref)
+    if M > 256:
+        y2, qy2, sy2 = fb.fp8_block_gemm_quant(*args, want_y=False)
+        torch.cuda.synchronize()
+        assert y2 is None
+        assert torch.equal(qy2, qy) and torch.equal(sy2, sy)

@@ -1,33 +1,36 @@
 #!/usr/bin/env python
 """Benchmark of the fine-grained FP8 linear-layer path on B200.
 
-One step = one pass of the whole path over the decode-shaped Llama-3-8B
-linears ((N, K) = QKV (6144, 4096), O (4096, 4096), gate+up (28672, 4096),
-down (4096, 14336); tokens M in {1, 8, 32, 128}):
+One pass of the path covers the decode-shaped Llama-3-8B linears ((N, K) =
+QKV (6144, 4096), O (4096, 4096), gate+up (28672, 4096), down (4096, 14336);
+tokens M in {1, 8, 32, 128}):
 
   1. weight quantization of the four bf16 weights (128x128 blocks)
   2. 2:4 prune + compress of the four weights
   3. for each M: the four activation quantizations (1x128 groups), the four
      dense block-scaled GEMMs, the four 2:4 sparse block-scaled GEMMs
 
-The metric is HBM throughput of the step (algorithmic bytes of every launch /
-device time), with the dominant kernel's roofline fraction against the
-measured copy bandwidth. Inputs are seeded synthetic bf16 tensors; the
-per-step working set (~2.7 GB) is far larger than L2 and every weight is
-re-read only after more than L2's worth of other traffic. The step is
-captured once as a CUDA graph and replayed, so host launch cost stays out of
-the device timing; the last steps of the timed region use copies of the graph
-with an event wherever the launch kind changes, for the per-kernel split.
+The metric is HBM throughput (algorithmic bytes of every launch / device
+time), with the dominant kernel's roofline fraction against the measured copy
+bandwidth. Inputs are seeded synthetic bf16 tensors; the per-pass working set
+(~2.7 GB) is far larger than L2 and every weight is re-read only after more
+than L2's worth of other traffic. A pass is captured once as a CUDA graph and
+replayed. A counted step is `passes` replays of that graph, with `passes`
+chosen so that the timed region lasts at least about a second whatever
+--steps says (the clock record and the per-kernel split then rest on many
+samples); the last passes of the timed region use copies of the graph with an
+event wherever the launch kind changes, for the live per-kernel split.
 
-The same JSON line also carries a "prefill" section: the dense GEMM on the
-prefill-shaped linears (M in {2048, 8192}, the four Llama-3-8B linears and
-the LM head) and the 2:4 GEMM at M = 4096, in TFLOP/s against the dense FP8
-tensor peak.
+The same JSON line also carries a "prefill" section (the dense GEMM on the
+prefill-shaped linears, M in {2048, 8192}, the four Llama-3-8B linears and the
+LM head; the 2:4 GEMM at M = 4096, in TFLOP/s against the dense FP8 tensor
+peak) and a "quantize" section (the quantizers at bandwidth-bound sizes, in
+GB/s against the copy bandwidth).
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU (replicas, weak scaling; no collective on the data path):
-  python -m torch.distributed.run --nnodes=1 --nproc-per-node N \
+  python -m torch.distributed.run --nnodes=1 --nproc-per-node N \\
       --master-addr 127.0.0.1 --master-port P bench.py --gpus N
 """
 
@@ -35,6 +38,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -54,9 +58,14 @@ WORKLOAD = "decode-shaped Llama-3-8B linears, M in {1,8,32,128}"
 LINEARS = ((6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336))
 TOKENS = (1, 8, 32, 128)
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+MIN_TIMED_S = 1.2          # the timed region lasts at least this long
 KERNELS = ("quant_weight", "prune24", "quant_act", "dense_gemm", "sparse_gemm")
 # Rows of the path the step runs.
 ROWS = KERNELS
+# The oracle's bounded sample of a pass: every weight row, and the token rows
+# for these M only.
+ORACLE_SAMPLE_M = (1, 8)
 
 
 # ----------------------------------------------------------------- bytes --
@@ -79,7 +88,7 @@ def kernel_bytes(kind, M, N, K):
 
 
 def step_launches():
-    """(kind, M, N, K) of every launch of one step, in issue order: the weight
+    """(kind, M, N, K) of every launch of one pass, in issue order: the weight
     rows, then per token count M the four activation quantizations, the four
     dense GEMMs and the four 2:4 GEMMs (same-kind launches back to back, so
     the live per-kernel split needs an event only where the kind changes)."""
@@ -95,10 +104,27 @@ def step_bytes():
     return sum(kernel_bytes(*l) for l in step_launches())
 
 
+def oracle_sample_launches():
+    """The launches of a pass the CPU oracle runs as its bounded sample."""
+    return [l for l in step_launches()
+            if l[0] in ("quant_weight", "prune24") or l[1] in ORACLE_SAMPLE_M]
+
+
+def bench_config(world, passes):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": WORKLOAD, "rows": list(ROWS), "linears_NK": [list(l) for l in LINEARS],
+            "tokens_M": list(TOKENS), "global_batch": sum(TOKENS) * passes * world,
+            "passes_per_step": passes, "pass_bytes": step_bytes(),
+            "launches_per_pass": len(step_launches()),
+            "parallelism": f"replicas x{world} (token data parallel, no collective)",
+            "l2": "working set per pass ~2.7 GB >> 126 MB L2; every weight is re-read only "
+                  "after >126 MB of other traffic; CUDA-graph replay"}
+
+
 # ------------------------------------------------------------ GPU step --
 
 class Step:
-    """Device buffers of one step and the launches through the C ABI."""
+    """Device buffers of one pass and the launches through the C ABI."""
 
     def __init__(self, device, seed=0):
         from fp8_block_scaled_group128_b200 import synth
@@ -130,7 +156,7 @@ class Step:
                 self.ys[(M, N, K)] = e(M, N, dt=torch.bfloat16)
 
     def launches(self):
-        """(kind, thunk) for every launch of one step, in issue order."""
+        """(kind, thunk) for every launch of one pass, in issue order."""
         from fp8_block_scaled_group128_b200 import binding as fb
         out = []
         for N, K in LINEARS:
@@ -155,7 +181,7 @@ class Step:
         return [(k, f) for k, f in out if k in ROWS]
 
     def run(self):
-        """Issue one step eagerly on the current stream."""
+        """Issue one pass eagerly on the current stream."""
         for _, f in self.launches():
             f()
 
@@ -164,8 +190,6 @@ class Step:
         return ({k: v.cpu().pin_memory() for k, v in self.w.items()},
                 {k: v.cpu().pin_memory() for k, v in self.x.items()})
 
-
-# --------------------------------------------------------------- clocks --
 
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons
@@ -259,8 +283,9 @@ def source_hash():
 
 
 def recorded_traffic(kind):
-    """Per-launch DRAM bytes of `kind` on this workload from the committed ncu
-    summary, or None if absent or taken on different kernel sources."""
+    """DRAM bytes / algorithmic bytes of `kind`, from the committed per-kernel
+    ncu captures (one kernel, a few launches each), or None if absent or
+    taken on different kernel sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -270,7 +295,9 @@ def recorded_traffic(kind):
     if d.get("source_hash") != source_hash():
         return None
     v = d.get("kernels", {}).get(kind)
-    return None if v is None else float(v["dram_bytes_per_launch"])
+    if v is None:
+        return None
+    return float(v["dram_bytes"]) / float(v["algorithmic_bytes"])
 
 
 def dist_info():
@@ -297,7 +324,19 @@ def barrier(world):
         dist.barrier()
 
 
-# ------------------------------------------------------------- prefill --
+def passes_per_step(steps, pass_ms):
+    """Graph replays per counted step so that `steps` steps last at least
+    MIN_TIMED_S."""
+    return max(1, math.ceil(MIN_TIMED_S * 1e3 / (max(steps, 1) * max(pass_ms, 1e-3))))
+
+
+def copies_beyond_l2(bytes_per_copy, cap=16):
+    """Input copies to rotate over so that back-to-back launches never find
+    their inputs in L2 (working set at least twice the L2 size)."""
+    return max(1, min(cap, math.ceil(2 * L2_BYTES / max(bytes_per_copy, 1))))
+
+
+# ------------------------------------------------- prefill and quantize --
 
 def fp8_tensor_peak():
     """Dense FP8 tensor peak (TFLOP/s): the measured cuBLAS bf16 burst figure
@@ -310,16 +349,43 @@ def fp8_tensor_peak():
         return 2.0 * 1590.0, "fallback bf16 1.59 PF/s x 2"
 
 
-def run_prefill(dev, stream, world, reps=10):
+def _time_graph(fns, stream, world, reps):
+    """Mean device time (ms) of one call, from a CUDA graph of `reps` calls
+    that cycle through `fns` (one warm-up replay, three timed; CUDA events on
+    the launching stream; max over ranks)."""
+    from fp8_block_scaled_group128_b200 import binding as fb
+    with torch.cuda.stream(stream):
+        for f in fns:
+            f()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps):
+            fns[i % len(fns)]()
+    with torch.cuda.stream(stream):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(3):
+            g.replay()
+        e1.record()
+    stream.synchronize()
+    assert fb.get_device_error(stream) == 0
+    del g
+    return max_over_ranks(e0.elapsed_time(e1) / (3 * reps), world)
+
+
+def run_prefill(dev, stream, world, reps=12):
     """Prefill-shaped GEMMs timed on their own: the dense GEMM at M in {2048,
     8192} on the four Llama-3-8B linears and the LM head, the 2:4 GEMM at
     M = 4096 on its two shapes, and on the down projection at M = 8192 the GEMM
     with the next layer's 1x128 quantization fused into its epilogue
     ("fused", codes only) against the GEMM followed by the activation
-    quantizer ("separate"). Each shape's launches are replayed from a CUDA
-    graph of `reps` back-to-back launches (one warm-up replay, three timed),
-    CUDA events on the launching stream. Inputs: the seeded synthetic llama
-    tensors, quantized / compressed on the device before timing."""
+    quantizer ("separate"). Each shape rotates over enough copies of its
+    quantized inputs that back-to-back launches find none of them in L2.
+    Inputs: the seeded synthetic llama tensors, quantized / compressed on the
+    device before timing."""
     from fp8_block_scaled_group128_b200 import binding as fb
     from fp8_block_scaled_group128_b200 import synth
     peak, peak_src = fp8_tensor_peak()
@@ -328,105 +394,158 @@ def run_prefill(dev, stream, world, reps=10):
     shapes += [("sparse", 4096, N, K) for N, K in synth.SPARSE_LINEARS]
     shapes += [(kind, 8192, 4096, 14336) for kind in ("fused", "separate")]
     rows, tot_flop, tot_ms = [], 0.0, 0.0
-    wcache = {}
     for kind, M, N, K in shapes:
         with torch.cuda.stream(stream):
-            key = (kind == "sparse", N, K)
-            if key not in wcache:
-                wcache.clear()
-                w = synth.weights("llama", N, K, seed=7).to(dev)
-                wcache[key] = (fb.prune24_compress(w)[:3] if kind == "sparse"
-                               else fb.fp8_quant_weight_block128(w))
-                del w
+            w = synth.weights("llama", N, K, seed=7).to(dev)
+            wq = fb.prune24_compress(w)[:3] if kind == "sparse" else fb.fp8_quant_weight_block128(w)
+            del w
             x = synth.activations("llama", M, K, seed=7).to(dev)
             qa, sa = fb.fp8_quant_act_group128(x)
+            del x
+            in_bytes = M * K + (N * K * 5 // 8 if kind == "sparse" else N * K)
+            n_cp = copies_beyond_l2(in_bytes, cap=8)
+            ins = [(qa.clone(), sa.clone(), [t.clone() for t in wq]) for _ in range(n_cp - 1)]
+            ins.append((qa, sa, list(wq)))
             y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-            wq = wcache[key]
             qy = torch.empty(M, N, dtype=torch.uint8, device=dev)
             sy = torch.empty(M, N // 128, dtype=torch.float32, device=dev)
+        fns = []
+        for a, s, wqq in ins:
             if kind == "dense":
-                fn = lambda: fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y)  # noqa: E731
+                fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_block_gemm(a, s, wqq[0], wqq[1], y=y))
             elif kind == "sparse":
-                fn = lambda: fb.fp8_sparse24_gemm(qa, sa, wq[0], wq[1], wq[2], y=y)  # noqa: E731
+                fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_sparse24_gemm(
+                    a, s, wqq[0], wqq[1], wqq[2], y=y))
             elif kind == "fused":
-                fn = lambda: fb.fp8_block_gemm_quant(  # noqa: E731
-                    qa, sa, wq[0], wq[1], qy=qy, sy=sy, want_y=False)
+                fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_block_gemm_quant(
+                    a, s, wqq[0], wqq[1], qy=qy, sy=sy, want_y=False))
             else:
-                fn = lambda: (fb.fp8_block_gemm(qa, sa, wq[0], wq[1], y=y),  # noqa: E731
-                              fb.fp8_quant_act_group128(y, qa=qy, sa=sy))
-            fn()
-        stream.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(reps):
-                fn()
-        with torch.cuda.stream(stream):
-            g.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record()
-            for _ in range(3):
-                g.replay()
-            e1.record()
-        stream.synchronize()
-        assert fb.get_device_error(stream) == 0
-        ms = max_over_ranks(e0.elapsed_time(e1) / (3 * reps), world)
+                fns.append(lambda a=a, s=s, wqq=wqq: (
+                    fb.fp8_block_gemm(a, s, wqq[0], wqq[1], y=y),
+                    fb.fp8_quant_act_group128(y, qa=qy, sa=sy)))
+        ms = _time_graph(fns, stream, world, reps)
         # algorithmic FLOPs: 2MNK dense; MNK (the kept half) for 2:4
         flop = (1.0 if kind == "sparse" else 2.0) * M * N * K
         tf = flop / (ms * 1e-3) / 1e12
         rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
-                     "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4)})
+                     "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4), "input_copies": n_cp})
         if kind == "dense":
             tot_flop += flop
             tot_ms += ms
-        del g, x, qa, sa, y, qy, sy
-    wcache.clear()
-    torch.cuda.empty_cache()
+        del fns, ins, qa, sa, wq, y, qy, sy
+        torch.cuda.empty_cache()
     agg = tot_flop / (tot_ms * 1e-3) / 1e12
     return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
             "dense_achieved": round(agg, 1), "dense_frac": round(agg / peak, 4),
             "note": "dense: 2MNK FLOPs; 2:4: MNK FLOPs (nonzero work) against the dense peak; "
                     "fused / separate: the down projection with the next layer's 1x128 "
-                    "quantization in the epilogue / after it (not in dense_achieved)",
+                    "quantization in the epilogue / after it (not in dense_achieved); inputs "
+                    "rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
+
+
+QUANT_SHAPES = (("quant_act", 8192, 0, 14336), ("quant_act", 8192, 0, 4096),
+                ("quant_act", 2048, 0, 4096), ("quant_weight", 0, 128256, 4096),
+                ("quant_weight", 0, 28672, 4096), ("prune24", 0, 128256, 4096),
+                ("prune24", 0, 28672, 4096))
+
+
+def run_quantize(dev, stream, world, reps=12):
+    """The quantizers at bandwidth-bound sizes (prefill activations, the LM
+    head and gate+up weights), each rotating over enough input copies that no
+    launch finds its input in L2; GB/s of algorithmic bytes against the
+    measured copy bandwidth."""
+    from fp8_block_scaled_group128_b200 import binding as fb
+    from fp8_block_scaled_group128_b200 import synth
+    hbm, kind_src = measured_peaks()
+    rows = []
+    for kind, M, N, K in QUANT_SHAPES:
+        rows_in = M if kind == "quant_act" else N
+        n_cp = copies_beyond_l2(2 * rows_in * K, cap=8)
+        with torch.cuda.stream(stream):
+            if kind == "quant_act":
+                src = synth.activations("llama", M, K, seed=5).to(dev)
+            else:
+                src = synth.weights("llama", N, K, seed=5).to(dev)
+            ins = [src] + [src.clone() for _ in range(n_cp - 1)]
+            NB = -(-rows_in // 128)
+            if kind == "quant_act":
+                q = torch.empty(M, K, dtype=torch.uint8, device=dev)
+                s = torch.empty(M, K // 128, dtype=torch.float32, device=dev)
+                fns = [lambda t=t: fb.fp8_quant_act_group128(t, qa=q, sa=s) for t in ins]
+            elif kind == "quant_weight":
+                q = torch.empty(N, K, dtype=torch.uint8, device=dev)
+                s = torch.empty(NB, K // 128, dtype=torch.float32, device=dev)
+                fns = [lambda t=t: fb.fp8_quant_weight_block128(t, qw=q, sw=s) for t in ins]
+            else:
+                v = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+                m = torch.empty(N, K // 8, dtype=torch.uint8, device=dev)
+                s = torch.empty(NB, K // 128, dtype=torch.float32, device=dev)
+                fns = [lambda t=t: fb.prune24_compress(t, vals=v, meta=m, sw=s) for t in ins]
+        ms = _time_graph(fns, stream, world, reps)
+        gbs = kernel_bytes(kind, M, N, K) / (ms * 1e-3) / 1e9
+        rows.append({"kernel": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
+                     "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4), "input_copies": n_cp})
+        del fns, ins, src
+        torch.cuda.empty_cache()
+    return {"bound": "hbm", "unit": "GB/s", "peak": hbm,
+            "peak_source": f"{kind_src} copy bandwidth", "shapes": rows}
 
 
 # ------------------------------------------------------------ CPU side --
 
-def oracle_sample(budget_s=15.0):
-    """Time the CPU oracle on a bounded sample of the step: the O-projection
-    linear (4096 x 4096) through all five stages at M = 8. Returns
-    (GB/s, seconds, description, threads)."""
-    import numpy as np
-    import oracle
-    from fp8_block_scaled_group128_b200 import synth
-    try:
-        from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(limits=1)
-    except ImportError:  # pragma: no cover
-        limiter = None
-    N, K, M = 4096, 4096, 8
-    w = synth.weights("llama", N, K, seed=0)
-    x = synth.activations("llama", M, K, seed=0)
-    byts = sum(kernel_bytes(k, 0 if k in ("quant_weight", "prune24") else M,
-                            0 if k == "quant_act" else N, K) for k in ROWS)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        qw, sw = oracle.quant_weight_block128(w)
-        vals, meta, sws, _ = oracle.prune24_compress(w)
-        qa, sa = oracle.quant_act_group128(x)
-        y = oracle.block_gemm(qa, sa, qw, sw)
-        ys = oracle.sparse24_gemm(qa, sa, vals, meta, sws) if "sparse_gemm" in ROWS else None
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or reps >= 50:
-            break
-    del y, ys, np
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
-    desc = (f"O-proj linear N=K=4096 at M=8 through the step's stages "
-            f"({', '.join(ROWS)}), {reps} repetition(s), 1 thread")
-    return byts * reps / el / 1e9, el, desc, 1
+class OracleSample:
+    """The CPU oracle (C++, all host cores) on a bounded sample of a pass:
+    every weight row of the four linears and the token rows at M in
+    ORACLE_SAMPLE_M, with the same seeded inputs as the GPU pass. Inputs are
+    generated and widened to fp32 once, outside the timing."""
+
+    def __init__(self, seed=0):
+        import numpy as np
+        import oracle
+        from fp8_block_scaled_group128_b200 import synth
+        self.oracle = oracle
+        self.launches = oracle_sample_launches()
+        self.bytes = sum(kernel_bytes(*l) for l in self.launches)
+        self.w = {nk: synth.weights("llama", *nk, seed=seed).float().numpy() for nk in LINEARS}
+        self.x = {}
+        for M in ORACLE_SAMPLE_M:
+            for i, nk in enumerate(LINEARS):
+                self.x[(M,) + nk] = np.ascontiguousarray(
+                    synth.activations("llama", M, nk[1], seed=seed + 101 * i).float().numpy())
+        self.cores = oracle.threads()
+        self.desc = (f"every weight row of the four linears and the token rows at M in "
+                     f"{list(ORACLE_SAMPLE_M)} ({len(self.launches)} of the pass's "
+                     f"{len(step_launches())} launches, {self.bytes / 1e9:.3f} GB of algorithmic "
+                     f"traffic); C++ oracle on {self.cores} host threads")
+
+    def run(self):
+        o = self.oracle
+        qw, sp, qa = {}, {}, {}
+        for kind, M, N, K in self.launches:
+            nk = (N, K)
+            if kind == "quant_weight":
+                qw[nk] = o.quant_weight_block128(self.w[nk])
+            elif kind == "prune24":
+                sp[nk] = o.prune24_compress(self.w[nk])[:3]
+            elif kind == "quant_act":
+                qa[(M,) + nk] = o.quant_act_group128(self.x[(M,) + nk])
+            elif kind == "dense_gemm":
+                o.block_gemm(*qa[(M,) + nk], *qw[nk])
+            elif kind == "sparse_gemm":
+                o.sparse24_gemm(*qa[(M,) + nk], *sp[nk])
+
+    def time(self, budget_s):
+        """Repeat the sample for at least `budget_s` seconds (at least once);
+        returns (GB/s, seconds, repetitions)."""
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            self.run()
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+        return self.bytes * reps / el / 1e9, el, reps
 
 
 # ---------------------------------------------------------------- arms --
@@ -443,7 +562,7 @@ def run_ours(args, rank, world, local):
     step = Step(dev, seed=rank)
     stream = torch.cuda.Stream(dev)
     launches = step_launches()
-    per_step_launches = len(launches)
+    per_pass_launches = len(launches)
 
     # eager warm-up (also runs the one-time per-device setup of the library)
     with torch.cuda.stream(stream):
@@ -452,14 +571,13 @@ def run_ours(args, rank, world, local):
     stream.synchronize()
     assert fb.get_device_error(stream) == 0
 
-    # The step is captured as one CUDA graph and replayed (host launch cost
-    # stays out of the device timing). The last R steps of the timed region
-    # replay copies of the graph that also hold an event record node wherever
-    # the launch kind changes (external events; each copy its own events):
-    # every kind's device time over those R steps is measured live inside the
-    # timed region, a run of same-kind launches as one span. Event nodes cost
-    # a few microseconds each, so the other steps run the plain graph.
-    R = min(10, args.steps)
+    # A pass is captured as one CUDA graph and replayed (host launch cost stays
+    # out of the device timing). The last R passes of the timed region replay
+    # copies of the graph that also hold an event record node wherever the
+    # launch kind changes (external events; each copy its own events): every
+    # kind's device time over those R passes is measured live inside the timed
+    # region, a run of same-kind launches as one span. Event nodes cost a few
+    # microseconds each, so the other passes run the plain graph.
     launches_fns = step.launches()
     # (kind, index of the first launch, index past the last) of each run
     groups = []
@@ -484,23 +602,34 @@ def run_ours(args, rank, world, local):
         return g, evs
 
     plain, _ = capture(False)
-    evented = [capture(True) for _ in range(R)]
-    stream.synchronize()
+    # graph warm-up, which also sizes the counted step
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             plain.replay()
+        t0.record()
+        for _ in range(5):
+            plain.replay()
+        t1.record()
+    stream.synchronize()
+    pass_ms = max_over_ranks(t0.elapsed_time(t1) / 5, world)
+    passes = passes_per_step(args.steps, pass_ms)
+    total_passes = passes * args.steps
+    R = min(10, total_passes)
+    evented = [capture(True) for _ in range(R)]
+    stream.synchronize()
+    with torch.cuda.stream(stream):
         for g, _ in evented:
             g.replay()
     torch.cuda.synchronize()
 
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     with ClockSampler(local) as clocks:
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             t0.record()
-            for _ in range(args.steps - R):
+            for _ in range(total_passes - R):
                 plain.replay()
             for g, _ in evented:
                 g.replay()
@@ -516,7 +645,7 @@ def run_ours(args, rank, world, local):
     ms_step = max_over_ranks(total_ms / args.steps, world)
 
     sb = step_bytes()
-    value = sb * world / (ms_step * 1e-3) / 1e9
+    value = sb * passes * world / (ms_step * 1e-3) / 1e9
     hbm_peak, peak_kind = measured_peaks()
 
     breakdown = {}
@@ -524,21 +653,26 @@ def run_ours(args, rank, world, local):
         kb = sum(kernel_bytes(*l) for l in launches if l[0] == k)
         n = sum(1 for l in launches if l[0] == k)
         ms = kernel_ms[k]
-        breakdown[k] = {"launches": n, "ms": round(ms, 4),
-                        "GB/s": round(kb / (ms * 1e-3) / 1e9, 1) if ms > 0 else None}
+        breakdown[k] = {"launches_per_pass": n, "ms_per_pass": round(ms, 4),
+                        "GB/s": round(kb / (ms * 1e-3) / 1e9, 1) if ms > 0 else None,
+                        "frac": round(kb / (ms * 1e-3) / 1e9 / hbm_peak, 4) if ms > 0 else None}
     dominant = max(ROWS, key=lambda k: kernel_ms[k])
     dom_launches = [l for l in launches if l[0] == dominant]
     dom_bytes_per_launch = sum(kernel_bytes(*l) for l in dom_launches) / len(dom_launches)
     dom_ms_per_launch = kernel_ms[dominant] / len(dom_launches)
     achieved = dom_bytes_per_launch / (dom_ms_per_launch * 1e-3) / 1e9
-    traffic = recorded_traffic(dominant)
+    ratio = recorded_traffic(dominant)
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
                 "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                 "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
-                "traffic": traffic}
+                "algorithmic_bytes_per_launch": round(dom_bytes_per_launch),
+                "traffic": None if ratio is None else round(ratio * dom_bytes_per_launch),
+                "traffic_source": "profiles/traffic.json: DRAM bytes / algorithmic bytes of "
+                                  "per-kernel ncu captures, times the algorithmic bytes per "
+                                  "launch" if ratio is not None else "no capture on these sources"}
 
-    # end to end: pinned host inputs -> device, the step through the C ABI,
+    # end to end: pinned host inputs -> device, one pass through the C ABI,
     # device -> host read of every output Y
     h_w, h_x = step.host_inputs()
     h2d = sum(t.numel() * t.element_size() for t in h_w.values()) + \
@@ -573,7 +707,8 @@ def run_ours(args, rank, world, local):
     stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": round(sb * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": UNIT,
-           "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "ms_per_step": round(e2e_ms, 3), "passes_per_step": 1,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
@@ -581,53 +716,59 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 x e4m3 -> fp32 accumulate, bf16 out",
         "data": "synthetic (seeded bf16, Llama-3-8B linear shapes)",
-        "config": {"workload": WORKLOAD, "rows": list(ROWS), "linears_NK": [list(l) for l in LINEARS],
-                   "tokens_M": list(TOKENS), "global_batch": sum(TOKENS) * world,
-                   "step_bytes": sb, "launches_per_step": per_step_launches,
-                   "event_nodes_per_evented_step": len(groups) + 1,
-                   "parallelism": f"replicas x{world} (token data parallel, no collective)",
-                   "l2": "working set per step ~2.7 GB >> 126 MB L2; every weight is re-read "
-                         "only after >126 MB of other traffic; CUDA-graph replay"},
+        "config": bench_config(world, passes),
+        "timed_region_s": round(total_ms * 1e-3, 3),
         "roofline": roofline,
         "kernels": breakdown,
         "e2e": e2e,
-        "gpu_launches": per_step_launches * args.steps,
+        "gpu_launches": per_pass_launches * total_passes,
         "clocks": clocks.summary(),
     }
-    if not args.no_prefill:
+    if not args.no_sections:
+        result["quantize"] = run_quantize(dev, stream, world)
         result["prefill"] = run_prefill(dev, stream, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, el, desc, cores = oracle_sample(args.cpu_budget)
-        result["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": cores,
-                                  "kind": "oracle", "sample": desc, "seconds": round(el, 2)}
+        sample = OracleSample(seed=0)
+        sample.run()   # first touch of the oracle's buffers, untimed
+        v, el, reps = sample.time(args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": sample.cores,
+                                  "kind": "oracle", "sample": f"{sample.desc}; {reps} repetition(s)",
+                                  "seconds": round(el, 2)}
     del plain, evented
     return result
 
 
 def run_reference(args, rank, world):
-    """The oracle (numpy, fp64 GEMM) on the host cores, bounded samples."""
+    """The oracle as it stands (C++, fp64 GEMM, every host core) on the host:
+    each counted step is one run of the bounded sample of a pass, timed by the
+    host clock. Rank 0 alone runs; other ranks return without work."""
     if rank != 0:
         return None
-    samples = []
-    for _ in range(max(0, args.warmup)):
-        oracle_sample(budget_s=0.0)
-    t0 = time.perf_counter()
+    sample = OracleSample(seed=0)
+    for _ in range(max(1, args.warmup)):
+        sample.run()
+    times = []
+    t_all = time.perf_counter()
     for _ in range(args.steps):
-        v, el, desc, cores = oracle_sample(budget_s=min(args.cpu_budget, 10.0))
-        samples.append(v)
-    el_all = time.perf_counter() - t0
-    v = statistics.mean(samples)
-    sb = step_bytes()
-    ms = sb / (v * 1e9) * 1e3
+        t0 = time.perf_counter()
+        sample.run()
+        times.append(time.perf_counter() - t0)
+    wall = time.perf_counter() - t_all
+    ms = 1e3 * wall / max(args.steps, 1)
+    v = sample.bytes * args.steps / wall / 1e9
+    cfg = bench_config(world, 1)
+    cfg["sample"] = sample.desc
+    cfg["sample_bytes"] = sample.bytes
     return {
         "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64 oracle (fp32 quantization arithmetic)",
-        "data": "synthetic (seeded bf16)",
-        "config": {"workload": WORKLOAD, "sample": desc, "wall_s": round(el_all, 1)},
-        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "vs_baseline": None, "dtype": "C++ oracle: fp32 quantization arithmetic, fp64 GEMM",
+        "data": "synthetic (seeded bf16, Llama-3-8B linear shapes)",
+        "config": cfg, "timed_region_s": round(wall, 2),
+        "step_s_min_max": [round(min(times), 3), round(max(times), 3)],
+        "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": sample.cores,
+                         "kind": "oracle", "sample": sample.desc},
         "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -642,8 +783,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true",
-                    help="skip the prefill-shaped GEMM section of the JSON line")
+    ap.add_argument("--no-sections", action="store_true",
+                    help="skip the prefill and quantize sections of the JSON line")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

@@ -3,13 +3,18 @@
     python -m fp8_block_scaled_group128_b200.build [--force]
 
 Each .cu file under csrc/ is compiled by nvcc in parallel to an object file
-under _build/, then linked into ``libfp8bs.so`` next to this file. Nothing is
-rebuilt when no source or header is newer than the library.
+under _build/, then linked into ``libfp8bs.so`` next to this file. The
+library is rebuilt whenever the SHA-256 of its sources, headers, this script
+and the compiler flags differs from the one recorded beside it
+(``libfp8bs.so.stamp``); file times play no part, so a library copied to
+another machine with its sources is reused only if it was built from exactly
+those sources.
 """
 
 import argparse
 import concurrent.futures as cf
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -20,6 +25,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfp8bs.so")
+STAMP = LIB + ".stamp"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -44,11 +50,23 @@ def _deps():
             + glob.glob(os.path.join(ROOT, "include", "*.h")) + [__file__])
 
 
+def source_digest():
+    """SHA-256 over every source and header (by name and content), this
+    script and the compiler flags."""
+    h = hashlib.sha256()
+    for d in sorted(_deps()):
+        h.update(os.path.relpath(d, ROOT).encode() + b"\0")
+        with open(d, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()
+
+
 def up_to_date():
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in _deps())
+    with open(STAMP) as f:
+        return f.read().strip() == source_digest()
 
 
 def _compile(src):
@@ -77,6 +95,8 @@ def build(force=False, verbose=False):
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link failed")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(source_digest() + "\n")
     return LIB
 
 

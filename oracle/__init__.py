@@ -1,24 +1,36 @@
 """CPU oracle for the fine-grained (block-scaled, group-128) FP8 linear layer.
 
 TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
-``cpu_baseline`` leg of ``bench.py`` may import this package; the library in
-``fp8_block_scaled_group128_b200`` never does, and shares no code with it.
+``cpu_baseline`` leg / reference arm of ``bench.py`` may import this package;
+the library in ``fp8_block_scaled_group128_b200`` never does, and shares no
+code with it.
 
-Everything is plain numpy, with floating point in fp64 except where the method
-fixes fp32 (the scale and the element division, see ``fp8_oracle``).
+Two statements of the same definitions, written separately:
+
+* ``fp8_oracle.cpp`` (plain C++17, double precision for the GEMM, fp32 where
+  the method fixes fp32: the scale and the element division; threaded over
+  independent outputs), reached through ``fp8_oracle_cpp`` -- the oracle the
+  GPU parity tests and the CPU baseline use, exported at package level;
+* ``fp8_oracle`` (numpy) -- the same arithmetic written a second time; the
+  CPU tests check both against the same pins and against each other.
 """
 
-from .fp8_oracle import (  # noqa: F401
+from . import fp8_oracle as numpy_oracle  # noqa: F401
+from . import fp8_oracle_cpp as cpp_oracle  # noqa: F401
+from .fp8_oracle_cpp import (  # noqa: F401
     E4M3_MAX,
     GROUP,
-    e4m3_encode,
+    bf16_ulp,
+    block_gemm,
+    decompress24,
     e4m3_decode,
+    e4m3_encode,
+    gemm_abs_sum,
+    gemm_error_bound,
+    prune24_compress,
     quant_act_group128,
     quant_weight_block128,
-    prune24_compress,
-    decompress24,
-    block_gemm,
+    set_threads,
     sparse24_gemm,
-    gemm_error_bound,
-    bf16_ulp,
+    threads,
 )

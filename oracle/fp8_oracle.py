@@ -1,8 +1,11 @@
 """Plain CPU oracle of the fine-grained FP8 linear layer (test infrastructure).
 
 This module is the slow, obviously-correct statement of what the layer
-computes. It is used only by the tests, the smoke check and the CPU baseline of
-the benchmark; the CUDA library never imports it and the two share no code.
+computes, written in numpy. The same definitions are written a second time in
+plain C++ (``fp8_oracle.cpp``), which is the oracle the GPU tests use; the CPU
+tests hold both to the same pins and to each other. Used only by the tests,
+the smoke check and the CPU baseline of the benchmark; the CUDA library never
+imports it and the two share no code.
 
 Sources (by page title and section):
 
@@ -343,14 +346,19 @@ def sparse24_gemm(qA, sA, vals, meta, sW, cols=None):
     return _gemm_rows(qA, sA, q_w, np.asarray(sW, np.float64)[n // GROUP])
 
 
+def gemm_abs_sum(qA, sA, qW, sW, cols=None):
+    """sum_k |a_k * w_k| per output, on the dequantized operands (fp64)."""
+    qA = np.asarray(qA, np.uint8)
+    q_w, s_w = _weight_rows(qW, sW, cols)
+    a = np.abs(e4m3_decode(qA)) * np.repeat(np.abs(np.asarray(sA, np.float64)), GROUP, axis=1)
+    w = np.abs(e4m3_decode(q_w)) * np.repeat(np.abs(s_w), GROUP, axis=1)
+    return a @ w.T
+
+
 def gemm_error_bound(qA, sA, qW, sW, cols=None, rel=1e-2):
     """Per-output tolerance rel * sum_k |a_k * w_k| on the dequantized
     operands (the test adds one bf16 ulp of the reference on top)."""
-    qA = np.asarray(qA, np.uint8)
-    q_w, s_w = _weight_rows(qW, sW, cols)
-    a = np.abs(e4m3_decode(qA)) * np.repeat(np.asarray(sA, np.float64), GROUP, axis=1)
-    w = np.abs(e4m3_decode(q_w)) * np.repeat(s_w, GROUP, axis=1)
-    return rel * (a @ w.T)
+    return rel * gemm_abs_sum(qA, sA, qW, sW, cols=cols)
 
 
 def bf16_ulp(y):

@@ -29,3 +29,11 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(params=["cpp", "numpy"], scope="session")
+def impl(request):
+    """Each statement of the oracle in turn: the C++ one (the oracle the GPU
+    tests use) and the numpy one. Every pin must hold for both."""
+    import oracle
+    return oracle.cpp_oracle if request.param == "cpp" else oracle.numpy_oracle

@@ -27,9 +27,31 @@ def to_dev(a, dtype=None):
     return t.contiguous().cuda()
 
 
-def check_gemm(y_gpu, y_ref, bound, label=""):
+def _dequant_abs(q, s_rows):
+    """|E4M3 value| x its scale, float64, with torch's own float8_e4m3fn decode
+    (a library routine, independent of the oracle); s_rows [rows, K/128]."""
+    v = torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).to(torch.float64).abs()
+    return v * torch.from_numpy(np.abs(np.asarray(s_rows, np.float64))).repeat_interleave(128, 1)
+
+
+def independent_abs_sum(qa, sa, qw, sw, cols=None):
+    """sum_k |a_k w_k| per output, computed here with one float64 matmul of
+    the dequantized magnitudes (weight row n uses scale row n // 128)."""
+    n = np.arange(qw.shape[0]) if cols is None else np.asarray(cols, np.int64)
+    a = _dequant_abs(qa, sa)
+    w = _dequant_abs(np.asarray(qw)[n], np.asarray(sw)[n // 128])
+    return (a @ w.T).numpy()
+
+
+def check_gemm(y_gpu, y_ref, operands, label="", cols=None):
     """The GEMM parity bar: |y - y_ref| <= 1e-2 * sum_k |a_k w_k| + 1 bf16 ulp
-    of the reference, on every compared output. Returns summary statistics."""
+    of the reference, on every compared output. `operands` = (qa, sa, qw, sw)
+    of the compared rows (qw, sw for all weight rows; `cols` picks the
+    compared ones). The oracle's bound is checked against sum |a w| computed
+    independently here. Returns summary statistics."""
+    bound = oracle.gemm_error_bound(*operands, cols=cols)
+    abs_sum = independent_abs_sum(*operands, cols=cols)
+    np.testing.assert_allclose(bound, 1e-2 * abs_sum, rtol=1e-9, atol=0.0)
     y = y_gpu.float().cpu().numpy().astype(np.float64)
     err = np.abs(y - y_ref)
     tol = bound + oracle.bf16_ulp(y_ref)
@@ -41,7 +63,7 @@ def check_gemm(y_gpu, y_ref, bound, label=""):
             f"gpu={y[tuple(i)]!r} ref={y_ref[tuple(i)]!r} tol={tol[tuple(i)]!r}")
     # error beyond the final bf16 rounding, relative to sum_k |a_k w_k|
     excess = np.maximum(err - 0.5 * oracle.bf16_ulp(y_ref), 0.0)
-    rel = excess / np.maximum(bound / 1e-2, 1e-300)
+    rel = excess / np.maximum(abs_sum, 1e-300)
     y_rn = torch.from_numpy(y_ref).to(torch.bfloat16).double().numpy()
     stats = {"label": label, "n": int(y.size),
              "max_err_over_sum": float(rel.max(initial=0.0)),

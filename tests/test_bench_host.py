@@ -55,6 +55,24 @@ def test_max_over_ranks_gloo_two_ranks():
     assert dict(out) == {0: 2.5, 1: 2.5}
 
 
+def test_counted_step_lasts_long_enough():
+    # 20 steps of a 0.75 ms pass: 80 passes per step (1.2 s); long passes: 1
+    assert bench.passes_per_step(20, 0.75) == 80
+    assert bench.passes_per_step(20, 0.75) * 20 * 0.75e-3 >= bench.MIN_TIMED_S
+    assert bench.passes_per_step(1000, 5.0) == 1
+    assert bench.copies_beyond_l2(16 << 20, cap=16) == 16
+    assert bench.copies_beyond_l2(1 << 30) == 1
+
+
+def test_oracle_sample_is_a_subset_of_the_pass():
+    s = bench.oracle_sample_launches()
+    assert set(s) <= set(bench.step_launches())
+    assert {l[0] for l in s} == set(bench.ROWS)
+    assert all(l[1] in bench.ORACLE_SAMPLE_M for l in s if l[0] not in ("quant_weight", "prune24"))
+    cfg = bench.bench_config(1, 3)
+    assert cfg["passes_per_step"] == 3 and cfg["global_batch"] == 3 * sum(bench.TOKENS)
+
+
 def test_clock_summary_parses_reasons():
     c = bench.ClockSampler(0)
     c.out = io.StringIO(
@@ -74,7 +92,8 @@ def test_recorded_traffic_requires_matching_sources(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
     h = bench.source_hash()
     (tmp_path / "profiles" / "traffic.json").write_text(
-        '{"source_hash": "%s", "kernels": {"prune24": {"dram_bytes_per_launch": 123}}}' % h)
-    assert bench.recorded_traffic("prune24") == 123.0
+        '{"source_hash": "%s", "kernels": {"prune24": {"dram_bytes": 123, '
+        '"algorithmic_bytes": 246}}}' % h)
+    assert bench.recorded_traffic("prune24") == 0.5
     (csrc / "a.cu").write_text("changed")
     assert bench.recorded_traffic("prune24") is None

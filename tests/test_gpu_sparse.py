@@ -52,8 +52,8 @@ def _sparse_case(kind, M, N, K, seed=0, rows=None, blocks=None, w=None, x=None):
     np.testing.assert_array_equal(sw_d[torch.from_numpy(nbs).cuda()].cpu().numpy().view(np.uint32),
                                   s_r.view(np.uint32))
     y_ref = oracle.sparse24_gemm(qa_r, sa_r, v_r, m_r, s_r)
-    bound = oracle.gemm_error_bound(qa_r, sa_r, oracle.decompress24(v_r, m_r), s_r)
-    return check_gemm(y[rd][:, nd], y_ref, bound, f"sparse {kind} M={M} N={N} K={K}"), y
+    ops = (qa_r, sa_r, oracle.decompress24(v_r, m_r), s_r)
+    return check_gemm(y[rd][:, nd], y_ref, ops, f"sparse {kind} M={M} N={N} K={K}"), y
 
 
 def _blocks(N, k, seed):
@@ -88,9 +88,14 @@ def test_ragged_shapes(M, N, K):
     assert stats["max_err_over_sum"] < 1e-4
 
 
-def test_sparse_matches_dense_on_pruned_weights():
-    """Same pruned weights through the dense and the sparse GEMM on the GPU."""
-    M, N, K = 64, 4096, 4096
+@pytest.mark.parametrize("M,N,K", [(64, 4096, 4096), (16, 14336, 4096), (16, 4096, 14336),
+                                   (4096, 14336, 4096), (4096, 4096, 14336)])
+def test_sparse_and_dense_on_the_same_pruned_weights(M, N, K):
+    """The 2:4 configuration's comparison with dense on the same pruned W: the
+    GPU prunes W, quantizes the pruned bf16 W densely and runs both GEMMs;
+    each output is checked element by element against the oracle (the sparse
+    GEMM of the oracle's compression, and the dense GEMM of its quantization
+    of the pruned W, which must be the same numbers)."""
     x = synth.activations("llama", M, K, seed=4)
     w = synth.weights("llama", N, K, seed=4)
     xd, wd = to_dev(x), to_dev(w)
@@ -100,10 +105,26 @@ def test_sparse_matches_dense_on_pruned_weights():
     ys = fb.fp8_sparse24_gemm(qa, sa, vals, meta, sws)
     yd = fb.fp8_block_gemm(qa, sa, qw, sw)
     torch.cuda.synchronize()
+    assert fb.get_device_error() == 0
     assert torch.equal(sw, sws)
-    diff = (ys.float() - yd.float()).abs()
-    scale = yd.float().abs().clamp_min(1e-30)
-    assert float((diff / scale).max()) <= 2 ** -7   # at most one bf16 rounding apart
+    NB = -(-N // 128)
+    rows = np.arange(M) if M <= 64 else _sample(M, 64, M, must=list(range(9, M, 128)) + [M - 1])
+    nbs = _blocks(N, 8 if M > 64 else 16, N + M)
+    n_idx = np.concatenate([np.arange(b * 128, min(N, b * 128 + 128)) for b in nbs])
+    qa_r, sa_r = oracle.quant_act_group128(x[torch.from_numpy(rows)])
+    v_r, m_r, s_r, wp_r = oracle.prune24_compress(w[torch.from_numpy(n_idx)])
+    qd_r, sd_r = oracle.quant_weight_block128(wp_r)
+    np.testing.assert_array_equal(qd_r, oracle.decompress24(v_r, m_r))
+    rd, nd = torch.from_numpy(rows).cuda(), torch.from_numpy(n_idx).cuda()
+    np.testing.assert_array_equal(wp[nd].float().cpu().numpy(), wp_r)
+    np.testing.assert_array_equal(qw[nd].cpu().numpy(), qd_r)
+    y_ref = oracle.sparse24_gemm(qa_r, sa_r, v_r, m_r, s_r)
+    np.testing.assert_array_equal(y_ref, oracle.block_gemm(qa_r, sa_r, qd_r, sd_r))
+    ops = (qa_r, sa_r, qd_r, sd_r)
+    st_s = check_gemm(ys[rd][:, nd], y_ref, ops, f"2:4 vs dense, sparse M={M} N={N} K={K}")
+    st_d = check_gemm(yd[rd][:, nd], y_ref, ops, f"2:4 vs dense, dense M={M} N={N} K={K}")
+    assert st_s["max_err_over_sum"] < 1e-4 and st_d["max_err_over_sum"] < 1e-4
+    assert NB > 0
 
 
 def test_ties_and_zero_groups():

@@ -9,7 +9,7 @@ import oracle
 from fp8_block_scaled_group128_b200 import synth
 
 
-def test_hand_computed_two_by_two():
+def test_hand_computed_two_by_two(impl):
     # K = 256 (two K-blocks), M = N = 2.
     qa = np.zeros((2, 256), np.uint8)
     qa[0, :128] = 0x38            # 1.0
@@ -20,58 +20,58 @@ def test_hand_computed_two_by_two():
     qw[0, :] = 0x38               # 1.0 everywhere
     qw[1, 128:] = 0x30            # 0.5 in the second K-block only
     sw = np.array([[1.0, 2.0]], np.float32)
-    y = oracle.block_gemm(qa, sa, qw, sw)
+    y = impl.block_gemm(qa, sa, qw, sw)
     # y00 = 0.5*1*(128*1*1) + 0.25*2*(128*2*1) = 64 + 128 = 192
     # y01 = 0 + 0.25*2*(128*2*0.5) = 64
     # y10 = 3*1*(-2*1) = -6 ; y11 = 0
     np.testing.assert_array_equal(y, np.array([[192.0, 64.0], [-6.0, 0.0]]))
 
 
-def test_ragged_n_uses_row_block_scales():
+def test_ragged_n_uses_row_block_scales(impl):
     # N = 130: rows 128, 129 take the second scale row.
     qa = np.full((1, 128), 0x38, np.uint8)
     sa = np.ones((1, 1), np.float32)
     qw = np.full((130, 128), 0x38, np.uint8)
     sw = np.array([[1.0], [0.5]], np.float32)
-    y = oracle.block_gemm(qa, sa, qw, sw)
+    y = impl.block_gemm(qa, sa, qw, sw)
     assert np.all(y[0, :128] == 128.0) and np.all(y[0, 128:] == 64.0)
-    y_cols = oracle.block_gemm(qa, sa, qw, sw, cols=[127, 128, 3])
+    y_cols = impl.block_gemm(qa, sa, qw, sw, cols=[127, 128, 3])
     np.testing.assert_array_equal(y_cols[0], [128.0, 64.0, 128.0])
 
 
-def test_exact_integer_case():
+def test_exact_integer_case(impl):
     rng = np.random.default_rng(2)
-    ints = np.array([oracle.e4m3_encode(np.array([v], np.float32))[0] for v in range(-16, 17)], np.uint8)
+    ints = np.array([impl.e4m3_encode(np.array([v], np.float32))[0] for v in range(-16, 17)], np.uint8)
     qa = rng.choice(ints, size=(5, 384))
     qw = rng.choice(ints, size=(7, 384))
     ones_a = np.ones((5, 3), np.float32)
     ones_w = np.ones((1, 3), np.float32)
-    y = oracle.block_gemm(qa, ones_a, qw, ones_w)
-    a = oracle.e4m3_decode(qa).astype(np.int64)
-    w = oracle.e4m3_decode(qw).astype(np.int64)
+    y = impl.block_gemm(qa, ones_a, qw, ones_w)
+    a = impl.e4m3_decode(qa).astype(np.int64)
+    w = impl.e4m3_decode(qw).astype(np.int64)
     np.testing.assert_array_equal(y, (a @ w.T).astype(np.float64))   # integer arithmetic
 
 
-def test_matches_dequantize_then_matmul_float64():
+def test_matches_dequantize_then_matmul_float64(impl):
     M, N, K = 9, 300, 640                 # ragged N, several K-blocks, M != N != K
     x = synth.activations("deepseek", M, K, seed=1)
     w = synth.weights("deepseek", N, K, seed=1)
-    qa, sa = oracle.quant_act_group128(x)
-    qw, sw = oracle.quant_weight_block128(w)
-    y = oracle.block_gemm(qa, sa, qw, sw)
+    qa, sa = impl.quant_act_group128(x)
+    qw, sw = impl.quant_weight_block128(w)
+    y = impl.block_gemm(qa, sa, qw, sw)
     # dequantize every element with its own scale, then one float64 matmul
-    a = torch.from_numpy(oracle.e4m3_decode(qa)) * torch.from_numpy(sa.astype(np.float64)).repeat_interleave(128, 1)
+    a = torch.from_numpy(impl.e4m3_decode(qa)) * torch.from_numpy(sa.astype(np.float64)).repeat_interleave(128, 1)
     sw_rows = torch.from_numpy(sw.astype(np.float64)).repeat_interleave(128, 0)[:N]
-    wd = torch.from_numpy(oracle.e4m3_decode(qw)) * sw_rows.repeat_interleave(128, 1)
+    wd = torch.from_numpy(impl.e4m3_decode(qw)) * sw_rows.repeat_interleave(128, 1)
     ref = (a @ wd.T).numpy()
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
     # and the quantized product approximates the bf16 product
     exact = (x.double() @ w.double().T).numpy()
-    bound = oracle.gemm_error_bound(qa, sa, qw, sw, rel=0.2)
+    bound = impl.gemm_error_bound(qa, sa, qw, sw, rel=0.2)
     assert np.all(np.abs(y - exact) <= bound + 1e-30)
 
 
-def test_power_of_two_scales_exact():
+def test_power_of_two_scales_exact(impl):
     rng = np.random.default_rng(3)
     qa = rng.integers(0, 256, size=(4, 256)).astype(np.uint8)
     qw = rng.integers(0, 256, size=(3, 256)).astype(np.uint8)
@@ -79,9 +79,9 @@ def test_power_of_two_scales_exact():
     qw[(qw & 0x7F) == 0x7F] = 0x38
     sa = np.exp2(rng.integers(-8, 8, size=(4, 2))).astype(np.float32)
     sw = np.exp2(rng.integers(-8, 8, size=(1, 2))).astype(np.float32)
-    y = oracle.block_gemm(qa, sa, qw, sw)
-    a = oracle.e4m3_decode(qa)
-    w = oracle.e4m3_decode(qw)
+    y = impl.block_gemm(qa, sa, qw, sw)
+    a = impl.e4m3_decode(qa)
+    w = impl.e4m3_decode(qw)
     want = np.zeros((4, 3))
     for m in range(4):
         for n in range(3):
@@ -90,20 +90,118 @@ def test_power_of_two_scales_exact():
     np.testing.assert_array_equal(y, want)   # every term and partial sum exact
 
 
-def test_sparse_equals_dense_on_pruned_weights():
+def test_sparse_equals_dense_on_pruned_weights(impl):
     x = synth.activations("llama", 6, 512, seed=8)
     w = synth.weights("llama", 260, 512, seed=8)
-    qa, sa = oracle.quant_act_group128(x)
-    vals, meta, sw, wp = oracle.prune24_compress(w)
-    qd, sd = oracle.quant_weight_block128(wp)
-    ys = oracle.sparse24_gemm(qa, sa, vals, meta, sw)
-    yd = oracle.block_gemm(qa, sa, qd, sd)
+    qa, sa = impl.quant_act_group128(x)
+    vals, meta, sw, wp = impl.prune24_compress(w)
+    qd, sd = impl.quant_weight_block128(wp)
+    ys = impl.sparse24_gemm(qa, sa, vals, meta, sw)
+    yd = impl.block_gemm(qa, sa, qd, sd)
     np.testing.assert_array_equal(ys, yd)
     cols = [0, 129, 259]
-    np.testing.assert_array_equal(oracle.sparse24_gemm(qa, sa, vals, meta, sw, cols=cols), yd[:, cols])
+    np.testing.assert_array_equal(impl.sparse24_gemm(qa, sa, vals, meta, sw, cols=cols), yd[:, cols])
 
 
-def test_bf16_ulp():
-    assert oracle.bf16_ulp(np.array([1.0]))[0] == 2.0 ** -7
-    assert oracle.bf16_ulp(np.array([-3.0]))[0] == 2.0 ** -6
-    assert oracle.bf16_ulp(np.array([0.0]))[0] == 2.0 ** -133
+def test_bf16_ulp(impl):
+    assert impl.bf16_ulp(np.array([1.0]))[0] == 2.0 ** -7
+    assert impl.bf16_ulp(np.array([-3.0]))[0] == 2.0 ** -6
+    assert impl.bf16_ulp(np.array([0.0]))[0] == 2.0 ** -133
+
+
+def _two_by_two_operands():
+    """The operands of test_hand_computed_two_by_two."""
+    qa = np.zeros((2, 256), np.uint8)
+    qa[0, :128] = 0x38            # 1.0
+    qa[0, 128:] = 0x40            # 2.0
+    qa[1, 0] = 0xC0               # -2.0
+    sa = np.array([[0.5, 0.25], [3.0, 7.0]], np.float32)
+    qw = np.zeros((2, 256), np.uint8)
+    qw[0, :] = 0x38
+    qw[1, 128:] = 0x30            # 0.5
+    sw = np.array([[1.0, 2.0]], np.float32)
+    return qa, sa, qw, sw
+
+
+def test_error_bound_hand_computed(impl):
+    """The parity tolerance rel * sum_k |a_k w_k| on hand-computed operands.
+    sum |a w|: y00 = 0.5*1*128 + 0.25*2*(128*2*1) = 192; y01 = 0.25*2*(128*2*0.5)
+    = 64; y10 = 3*1*|-2*1| = 6; y11 = 0 (row 1 meets only zero weights)."""
+    qa, sa, qw, sw = _two_by_two_operands()
+    np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, rel=1.0),
+                                  [[192.0, 64.0], [6.0, 0.0]])
+    # the default rel is the task's 1e-2
+    np.testing.assert_allclose(impl.gemm_error_bound(qa, sa, qw, sw),
+                               [[1.92, 0.64], [0.06, 0.0]], rtol=1e-15)
+    np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, cols=[1], rel=1.0),
+                                  [[64.0], [0.0]])
+
+
+def test_error_bound_counts_magnitudes_not_the_signed_sum(impl):
+    """Terms of opposite sign cancel in y but not in the bound: a = (+1 x 64,
+    -1 x 64), w = 1 gives y = 0 and sum |a w| = 128; a negative weight block
+    and a negative code change nothing."""
+    qa = np.zeros((1, 128), np.uint8)
+    qa[0, :64] = 0x38
+    qa[0, 64:] = 0xB8             # -1.0
+    qw = np.full((2, 128), 0x38, np.uint8)
+    qw[1] = 0xB8
+    sa = np.ones((1, 1), np.float32)
+    sw = np.array([[0.25]], np.float32)
+    np.testing.assert_array_equal(impl.block_gemm(qa, sa, qw, sw), [[0.0, 0.0]])
+    np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, rel=1.0), [[32.0, 32.0]])
+
+
+def test_error_bound_ragged_row_blocks(impl):
+    """N = 130: rows 128, 129 take the second scale row; K = 256 with
+    different block scales per K-block; sum |a w| = sum_kb 128 * |sa| * |sw|."""
+    qa = np.full((1, 256), 0x40, np.uint8)      # 2.0
+    sa = np.array([[1.0, 0.5]], np.float32)
+    qw = np.full((130, 256), 0xB0, np.uint8)    # -0.5
+    sw = np.array([[1.0, 4.0], [0.125, 8.0]], np.float32)
+    b = impl.gemm_error_bound(qa, sa, qw, sw, rel=1.0)
+    # rows < 128: 128*2*0.5*(1*1 + 0.5*4) = 384 ; rows 128, 129: 128*(0.125 + 0.5*8) = 528
+    assert np.all(b[0, :128] == 384.0) and np.all(b[0, 128:] == 528.0)
+    np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, cols=[129, 0], rel=1.0),
+                                  [[528.0, 384.0]])
+
+
+def test_cpp_and_numpy_statements_agree():
+    """The two statements of the oracle give the same codes, scales, metadata,
+    pruned weights and GEMM outputs, bit for bit, on every workload kind (and
+    bounds equal up to the summation order of sum |a w|)."""
+    import oracle
+    c, n = oracle.cpp_oracle, oracle.numpy_oracle
+    for kind, M, N, K, seed in (("tiny", 16, 256, 256, 0), ("llama", 33, 520, 1024, 1),
+                                ("deepseek", 9, 300, 640, 2)):
+        x = synth.activations(kind, M, K, seed=seed)
+        w = synth.weights(kind, N, K, seed=seed)
+        for f in ("quant_act_group128", "quant_weight_block128", "prune24_compress"):
+            arg = x if f == "quant_act_group128" else w
+            for a, b in zip(getattr(c, f)(arg), getattr(n, f)(arg)):
+                np.testing.assert_array_equal(np.asarray(a).view(np.uint8), np.asarray(b).view(np.uint8))
+        qa, sa = c.quant_act_group128(x)
+        qw, sw = c.quant_weight_block128(w)
+        vals, meta, sws, _ = c.prune24_compress(w)
+        np.testing.assert_array_equal(c.block_gemm(qa, sa, qw, sw), n.block_gemm(qa, sa, qw, sw))
+        np.testing.assert_array_equal(c.sparse24_gemm(qa, sa, vals, meta, sws),
+                                      n.sparse24_gemm(qa, sa, vals, meta, sws))
+        np.testing.assert_array_equal(c.decompress24(vals, meta), n.decompress24(vals, meta))
+        np.testing.assert_allclose(c.gemm_error_bound(qa, sa, qw, sw),
+                                   n.gemm_error_bound(qa, sa, qw, sw), rtol=1e-13)
+
+
+def test_cpp_oracle_result_does_not_depend_on_thread_count():
+    import oracle
+    x = synth.activations("llama", 5, 512, seed=3)
+    w = synth.weights("llama", 260, 512, seed=3)
+    qa, sa = oracle.quant_act_group128(x)
+    qw, sw = oracle.quant_weight_block128(w)
+    y_all = oracle.block_gemm(qa, sa, qw, sw)
+    try:
+        oracle.set_threads(1)
+        assert oracle.threads() == 1
+        np.testing.assert_array_equal(oracle.block_gemm(qa, sa, qw, sw), y_all)
+        np.testing.assert_array_equal(oracle.quant_weight_block128(w)[0], qw)
+    finally:
+        oracle.set_threads(0)

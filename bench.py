@@ -295,9 +295,10 @@ def recorded_traffic(kind):
     if d.get("source_hash") != source_hash():
         return None
     v = d.get("kernels", {}).get(kind)
-    if v is None:
+    try:
+        return float(v["dram_bytes"]) / float(v["algorithmic_bytes"])
+    except (TypeError, KeyError, ValueError, ZeroDivisionError):
         return None
-    return float(v["dram_bytes"]) / float(v["algorithmic_bytes"])
 
 
 def dist_info():

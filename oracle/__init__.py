@@ -22,15 +22,21 @@ from .fp8_oracle_cpp import (  # noqa: F401
     GROUP,
     bf16_ulp,
     block_gemm,
+    block_gemm_ue8m0,
     decompress24,
     e4m3_decode,
     e4m3_encode,
     gemm_abs_sum,
     gemm_error_bound,
+    gemm_error_bound_ue8m0,
     prune24_compress,
     quant_act_group128,
+    quant_act_group128_ue8m0,
     quant_weight_block128,
+    quant_weight_block128_ue8m0,
     set_threads,
     sparse24_gemm,
     threads,
+    ue8m0_decode,
+    ue8m0_of_amax,
 )

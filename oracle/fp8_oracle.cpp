@@ -147,6 +147,24 @@ uint8_t quantize_one(float x, float s) {
   return e4m3_encode(ratio);
 }
 
+// UE8M0 ("float8_e8m0fnu": 8 exponent bits, no sign, no mantissa): code c
+// stands for 2^(c - 127); 0xFF is NaN. The scale of a group or block is the
+// smallest power of two s with 448 * s >= amax, so no element saturates;
+// amax == 0 (and any amax below 448 * 2^-127) takes the smallest code, 0.
+int ue8m0_code_of_amax(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  int e = 0;
+  std::frexp(static_cast<double>(amax) / 448.0, &e);   // amax / 448 < 2^e (approximately)
+  // settle e exactly: 448 * 2^e >= amax and 448 * 2^(e-1) < amax
+  while (e > -127 && std::ldexp(448.0, e - 1) >= static_cast<double>(amax)) --e;
+  while (std::ldexp(448.0, e) < static_cast<double>(amax)) ++e;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e + 127;
+}
+
+float ue8m0_scale(int code) { return static_cast<float>(std::ldexp(1.0, code - 127)); }
+
 }  // namespace
 
 extern "C" {
@@ -268,6 +286,58 @@ void orc_decompress24(const uint8_t* vals, const uint8_t* meta, int64_t N, int64
       dst[i0] = vals[n * (K / 2) + 2 * g];
       dst[i1] = vals[n * (K / 2) + 2 * g + 1];
     }
+  });
+}
+
+// Value of UE8M0 scale codes as fp32 (2^(c - 127), exact; NaN for 0xFF).
+void orc_ue8m0_decode(const uint8_t* code, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = code[i] == 0xFF ? std::nanf("") : ue8m0_scale(code[i]);
+}
+
+// UE8M0 scale codes of the given amax values.
+void orc_ue8m0_of_amax(const float* amax, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = static_cast<uint8_t>(ue8m0_code_of_amax(amax[i]));
+}
+
+// The UE8M0 variant of the activation quantizer: per 1x128 group the scale
+// is the power of two 2^(c - 127) of ue8m0_code_of_amax(amax), stored as its
+// code sa8[m][g]; the elements are e4m3(fl32(x / s)) as before.
+void orc_quant_act_group128_ue8m0(const float* x, int64_t M, int64_t K, uint8_t* qa,
+                                  uint8_t* sa8) {
+  const int64_t KB = K / kGroup;
+  parallel_for(M, [&](int64_t m) {
+    for (int64_t g = 0; g < KB; ++g) {
+      const float* xg = x + m * K + g * kGroup;
+      float amax = 0.0f;
+      for (int i = 0; i < kGroup; ++i) amax = std::max(amax, std::fabs(xg[i]));
+      const int c = ue8m0_code_of_amax(amax);
+      sa8[m * KB + g] = static_cast<uint8_t>(c);
+      const float s = ue8m0_scale(c);
+      for (int i = 0; i < kGroup; ++i) qa[m * K + g * kGroup + i] = quantize_one(xg[i], s);
+    }
+  });
+}
+
+// The UE8M0 variant of the weight quantizer (128x128 blocks, ragged last row
+// block over its valid rows).
+void orc_quant_weight_block128_ue8m0(const float* w, int64_t N, int64_t K, uint8_t* qw,
+                                     uint8_t* sw8) {
+  const int64_t KB = K / kGroup, NB = (N + kGroup - 1) / kGroup;
+  parallel_for(NB * KB, [&](int64_t blk) {
+    const int64_t nb = blk / KB, kb = blk % KB;
+    const int64_t r0 = nb * kGroup, r1 = std::min<int64_t>(N, r0 + kGroup);
+    float amax = 0.0f;
+    for (int64_t r = r0; r < r1; ++r)
+      for (int i = 0; i < kGroup; ++i) amax = std::max(amax, std::fabs(w[r * K + kb * kGroup + i]));
+    const int c = ue8m0_code_of_amax(amax);
+    sw8[nb * KB + kb] = static_cast<uint8_t>(c);
+    const float s = ue8m0_scale(c);
+    for (int64_t r = r0; r < r1; ++r)
+      for (int i = 0; i < kGroup; ++i) {
+        const int64_t k = kb * kGroup + i;
+        qw[r * K + k] = quantize_one(w[r * K + k], s);
+      }
   });
 }
 

@@ -369,3 +369,75 @@ def bf16_ulp(y):
     e = np.maximum(ex - 1, -126)
     ulp = np.ldexp(1.0, e - 7)
     return np.where(y == 0, 2.0 ** -133, ulp)
+
+
+# ----------------------------------------------------------------------------
+# UE8M0 scale variant ("Format d'échelle UE8M0": scales stored as
+# float8_e8m0fnu, a bare power of two)
+# ----------------------------------------------------------------------------
+
+def ue8m0_decode(code):
+    """fp32 value 2^(c - 127) of each UE8M0 code (8 exponent bits, no sign,
+    no mantissa; 0xFF is NaN)."""
+    c = np.asarray(code, np.uint8).astype(np.int64)
+    v = np.ldexp(np.float64(1.0), c - 127).astype(np.float32)
+    return np.where(c == 255, np.float32(np.nan), v)
+
+
+def ue8m0_of_amax(amax):
+    """Code of the smallest power of two s with 448 * s >= amax (no element
+    of the group saturates), clamped to the codes 0..254; amax == 0 -> 0."""
+    a = np.asarray(amax, np.float32).astype(np.float64)
+    # candidate e from the binade of amax / 448, then settled exactly with
+    # the comparisons 448 * 2^e >= amax > 448 * 2^(e - 1)
+    _, e = np.frexp(np.where(a > 0, a / E4M3_MAX, 1.0))
+    e = e.astype(np.int64)
+    for _ in range(2):
+        e = np.where(np.ldexp(E4M3_MAX, e - 1) >= a, e - 1, e)
+    for _ in range(2):
+        e = np.where(np.ldexp(E4M3_MAX, e) < a, e + 1, e)
+    e = np.clip(e, -127, 127)
+    return np.where(a > 0, e + 127, 0).astype(np.uint8)
+
+
+def quant_act_group128_ue8m0(x):
+    """Per 1x128 group: code c = ue8m0_of_amax(amax), s = 2^(c - 127),
+    qA = e4m3(fl32(x / s)). Returns (qA [M, K], sA8 uint8 [M, K/128])."""
+    x32 = _as_f32(x)
+    M, K = x32.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    g = x32.reshape(M, K // GROUP, GROUP)
+    amax = np.abs(g).max(axis=2) if M * K else np.zeros((M, K // GROUP), np.float32)
+    sa8 = ue8m0_of_amax(amax)
+    qa = _quantize_with_scale(g, ue8m0_decode(sa8)[:, :, None]).reshape(M, K)
+    return qa, sa8
+
+
+def quant_weight_block128_ue8m0(w):
+    """Per 128x128 block (ragged last row block over its valid rows): the
+    same with the block amax. Returns (qW [N, K], sW8 uint8 [NB, KB])."""
+    w32 = _as_f32(w)
+    N, K = w32.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    NB, KB = -(-N // GROUP), K // GROUP
+    sw8 = np.zeros((NB, KB), np.uint8)
+    qw = np.zeros((N, K), np.uint8)
+    for nb in range(NB):
+        r0, r1 = nb * GROUP, min(N, (nb + 1) * GROUP)
+        for kb in range(KB):
+            blk = w32[r0:r1, kb * GROUP:(kb + 1) * GROUP]
+            c = ue8m0_of_amax(np.float32(np.abs(blk).max()))
+            sw8[nb, kb] = c
+            qw[r0:r1, kb * GROUP:(kb + 1) * GROUP] = _quantize_with_scale(blk, ue8m0_decode(c))
+    return qw, sw8
+
+
+def block_gemm_ue8m0(qA, sA8, qW, sW8, cols=None):
+    """The block-scaled GEMM with each scale the power of two of its code."""
+    return block_gemm(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols)
+
+
+def gemm_error_bound_ue8m0(qA, sA8, qW, sW8, cols=None, rel=1e-2):
+    return gemm_error_bound(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols, rel=rel)

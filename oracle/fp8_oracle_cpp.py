@@ -33,6 +33,10 @@ _SIGS = {
     "orc_block_gemm": (None, [_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_sparse24_gemm": (None, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_gemm_abs_sum": (None, [_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
+    "orc_ue8m0_decode": (None, [_P, _I64, _P]),
+    "orc_ue8m0_of_amax": (None, [_P, _I64, _P]),
+    "orc_quant_act_group128_ue8m0": (None, [_P, _I64, _I64, _P, _P]),
+    "orc_quant_weight_block128_ue8m0": (None, [_P, _I64, _I64, _P, _P]),
 }
 
 
@@ -190,3 +194,53 @@ def gemm_error_bound(qA, sA, qW, sW, cols=None, rel=1e-2):
     """Per-output tolerance rel * sum_k |a_k * w_k| (the test adds one bf16
     ulp of the reference on top)."""
     return rel * gemm_abs_sum(qA, sA, qW, sW, cols=cols)
+
+
+# ----------------------------------------------------------- UE8M0 scales --
+
+def ue8m0_decode(code):
+    """fp32 value 2^(c - 127) of each UE8M0 scale code (NaN for 0xFF)."""
+    c = _u8(code)
+    out = np.empty(c.shape, np.float32)
+    lib().orc_ue8m0_decode(_p(c), c.size, _p(out))
+    return out
+
+
+def ue8m0_of_amax(amax):
+    """UE8M0 code of the smallest power of two s with 448 * s >= amax."""
+    a = _f32(amax)
+    out = np.empty(a.shape, np.uint8)
+    lib().orc_ue8m0_of_amax(_p(a), a.size, _p(out))
+    return out
+
+
+def quant_act_group128_ue8m0(x):
+    """(qA uint8 [M, K], sA8 uint8 [M, K/128] UE8M0 codes)."""
+    x = _f32(x)
+    M, K = x.shape
+    _check_k(K)
+    qa = np.empty((M, K), np.uint8)
+    sa8 = np.empty((M, K // GROUP), np.uint8)
+    lib().orc_quant_act_group128_ue8m0(_p(x), M, K, _p(qa), _p(sa8))
+    return qa, sa8
+
+
+def quant_weight_block128_ue8m0(w):
+    """(qW uint8 [N, K], sW8 uint8 [ceil(N/128), K/128] UE8M0 codes)."""
+    w = _f32(w)
+    N, K = w.shape
+    _check_k(K)
+    qw = np.empty((N, K), np.uint8)
+    sw8 = np.empty((-(-N // GROUP), K // GROUP), np.uint8)
+    lib().orc_quant_weight_block128_ue8m0(_p(w), N, K, _p(qw), _p(sw8))
+    return qw, sw8
+
+
+def block_gemm_ue8m0(qA, sA8, qW, sW8, cols=None):
+    """The block-scaled GEMM with UE8M0 scales: the same formula, each scale
+    being the power of two its code stands for."""
+    return block_gemm(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols)
+
+
+def gemm_error_bound_ue8m0(qA, sA8, qW, sW8, cols=None, rel=1e-2):
+    return gemm_error_bound(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols, rel=rel)

@@ -176,8 +176,9 @@ def test_cpp_and_numpy_statements_agree():
                                 ("deepseek", 9, 300, 640, 2)):
         x = synth.activations(kind, M, K, seed=seed)
         w = synth.weights(kind, N, K, seed=seed)
-        for f in ("quant_act_group128", "quant_weight_block128", "prune24_compress"):
-            arg = x if f == "quant_act_group128" else w
+        for f in ("quant_act_group128", "quant_weight_block128", "prune24_compress",
+                  "quant_act_group128_ue8m0", "quant_weight_block128_ue8m0"):
+            arg = x if f.startswith("quant_act") else w
             for a, b in zip(getattr(c, f)(arg), getattr(n, f)(arg)):
                 np.testing.assert_array_equal(np.asarray(a).view(np.uint8), np.asarray(b).view(np.uint8))
         qa, sa = c.quant_act_group128(x)

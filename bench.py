@@ -23,9 +23,10 @@ event wherever the launch kind changes, for the live per-kernel split.
 
 The same JSON line also carries a "prefill" section (the dense GEMM on the
 prefill-shaped linears, M in {2048, 8192}, the four Llama-3-8B linears and the
-LM head; the 2:4 GEMM at M = 4096, in TFLOP/s against the dense FP8 tensor
-peak) and a "quantize" section (the quantizers at bandwidth-bound sizes, in
-GB/s against the copy bandwidth).
+LM head, with fp32 scales and with UE8M0 scales; the 2:4 GEMM at M = 4096; in
+TFLOP/s against the dense FP8 tensor peak), a "quantize" section (the
+quantizers at bandwidth-bound sizes, in GB/s against the copy bandwidth) and
+an "accuracy" section (both scale formats against the exact product).
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -379,34 +380,46 @@ def _time_graph(fns, stream, world, reps):
 
 def run_prefill(dev, stream, world, reps=12):
     """Prefill-shaped GEMMs timed on their own: the dense GEMM at M in {2048,
-    8192} on the four Llama-3-8B linears and the LM head, the 2:4 GEMM at
-    M = 4096 on its two shapes, and on the down projection at M = 8192 the GEMM
-    with the next layer's 1x128 quantization fused into its epilogue
-    ("fused", codes only) against the GEMM followed by the activation
-    quantizer ("separate"). Each shape rotates over enough copies of its
-    quantized inputs that back-to-back launches find none of them in L2.
-    Inputs: the seeded synthetic llama tensors, quantized / compressed on the
-    device before timing."""
+    8192} on the four Llama-3-8B linears and the LM head, with fp32 scales
+    ("dense") and with UE8M0 scales ("ue8m0", the tensor cores' block
+    scaling); the 2:4 GEMM at M = 4096 on its two shapes; and on the down
+    projection at M = 8192 the GEMM with the next layer's 1x128 quantization
+    fused into its epilogue ("fused", codes only) against the GEMM followed by
+    the activation quantizer ("separate"). Each shape rotates over enough
+    copies of its quantized inputs that back-to-back launches find none of
+    them in L2. Inputs: the seeded synthetic llama tensors, quantized /
+    compressed on the device before timing."""
     from fp8_block_scaled_group128_b200 import binding as fb
     from fp8_block_scaled_group128_b200 import synth
     peak, peak_src = fp8_tensor_peak()
-    shapes = [("dense", M, N, K) for M in synth.PREFILL_M
-              for N, K in synth.LLAMA3_8B_LINEARS + (synth.LLAMA3_8B_LM_HEAD,)]
+    shapes = [(kind, M, N, K) for N, K in synth.LLAMA3_8B_LINEARS + (synth.LLAMA3_8B_LM_HEAD,)
+              for M in synth.PREFILL_M for kind in ("dense", "ue8m0")]
     shapes += [("sparse", 4096, N, K) for N, K in synth.SPARSE_LINEARS]
     shapes += [(kind, 8192, 4096, 14336) for kind in ("fused", "separate")]
-    rows, tot_flop, tot_ms = [], 0.0, 0.0
+    rows, tot = [], {"dense": [0.0, 0.0], "ue8m0": [0.0, 0.0]}
+    wcache = {}
     for kind, M, N, K in shapes:
         with torch.cuda.stream(stream):
-            w = synth.weights("llama", N, K, seed=7).to(dev)
-            wq = fb.prune24_compress(w)[:3] if kind == "sparse" else fb.fp8_quant_weight_block128(w)
-            del w
+            key = (N, K)
+            if key not in wcache:
+                wcache.clear()
+                torch.cuda.empty_cache()
+                wcache[key] = synth.weights("llama", N, K, seed=7).to(dev)
+            w = wcache[key]
+            if kind == "sparse":
+                wq = list(fb.prune24_compress(w)[:3])
+            elif kind == "ue8m0":
+                wq = list(fb.fp8_quant_weight_block128_ue8m0(w))
+            else:
+                wq = list(fb.fp8_quant_weight_block128(w))
             x = synth.activations("llama", M, K, seed=7).to(dev)
-            qa, sa = fb.fp8_quant_act_group128(x)
+            qa, sa = (fb.fp8_quant_act_group128_ue8m0(x) if kind == "ue8m0"
+                      else fb.fp8_quant_act_group128(x))
             del x
             in_bytes = M * K + (N * K * 5 // 8 if kind == "sparse" else N * K)
             n_cp = copies_beyond_l2(in_bytes, cap=8)
             ins = [(qa.clone(), sa.clone(), [t.clone() for t in wq]) for _ in range(n_cp - 1)]
-            ins.append((qa, sa, list(wq)))
+            ins.append((qa, sa, wq))
             y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
             qy = torch.empty(M, N, dtype=torch.uint8, device=dev)
             sy = torch.empty(M, N // 128, dtype=torch.float32, device=dev)
@@ -414,6 +427,9 @@ def run_prefill(dev, stream, world, reps=12):
         for a, s, wqq in ins:
             if kind == "dense":
                 fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_block_gemm(a, s, wqq[0], wqq[1], y=y))
+            elif kind == "ue8m0":
+                fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_block_gemm_ue8m0(
+                    a, s, wqq[0], wqq[1], y=y))
             elif kind == "sparse":
                 fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_sparse24_gemm(
                     a, s, wqq[0], wqq[1], wqq[2], y=y))
@@ -430,19 +446,57 @@ def run_prefill(dev, stream, world, reps=12):
         tf = flop / (ms * 1e-3) / 1e12
         rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
                      "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4), "input_copies": n_cp})
-        if kind == "dense":
-            tot_flop += flop
-            tot_ms += ms
+        if kind in tot:
+            tot[kind][0] += flop
+            tot[kind][1] += ms
         del fns, ins, qa, sa, wq, y, qy, sy
-        torch.cuda.empty_cache()
-    agg = tot_flop / (tot_ms * 1e-3) / 1e12
+    wcache.clear()
+    torch.cuda.empty_cache()
+    agg = {k: v[0] / (v[1] * 1e-3) / 1e12 for k, v in tot.items()}
     return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
-            "dense_achieved": round(agg, 1), "dense_frac": round(agg / peak, 4),
-            "note": "dense: 2MNK FLOPs; 2:4: MNK FLOPs (nonzero work) against the dense peak; "
-                    "fused / separate: the down projection with the next layer's 1x128 "
-                    "quantization in the epilogue / after it (not in dense_achieved); inputs "
+            "dense_achieved": round(agg["dense"], 1), "dense_frac": round(agg["dense"] / peak, 4),
+            "ue8m0_achieved": round(agg["ue8m0"], 1), "ue8m0_frac": round(agg["ue8m0"] / peak, 4),
+            "note": "dense: fp32 scales (per-K-block promotion), 2MNK FLOPs; ue8m0: power-of-two "
+                    "scales applied by the block-scaled MMA; 2:4: MNK FLOPs (nonzero work) against "
+                    "the dense peak; fused / separate: the down projection with the next layer's "
+                    "1x128 quantization in the epilogue / after it (not in dense_achieved); inputs "
                     "rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
+
+
+def run_accuracy(dev):
+    """Accuracy of the two scale formats on prefill-shaped linears (the llama
+    QKV at M = 2048 and the DeepSeek-V3 (7168, 7168) linear at M = 4096):
+    relative Frobenius error and largest error / largest |y| of the GPU output
+    against the exact product of the bf16 inputs (float64 on the host), on 64
+    sampled token rows x 512 sampled output columns."""
+    import numpy as np
+    from fp8_block_scaled_group128_b200 import binding as fb
+    from fp8_block_scaled_group128_b200 import synth
+    out = []
+    for kind, M, N, K in (("llama", 2048, 6144, 4096), ("deepseek", 4096, 7168, 7168)):
+        x = synth.activations(kind, M, K, seed=11)
+        w = synth.weights(kind, N, K, seed=11)
+        rng = np.random.default_rng(M + N)
+        r = torch.from_numpy(np.sort(rng.choice(M, 64, replace=False)))
+        c = torch.from_numpy(np.sort(rng.choice(N, 512, replace=False)))
+        exact = x[r].double() @ w[c].double().T
+        xd, wd = x.to(dev), w.to(dev)
+        res = {"workload": kind, "M": M, "N": N, "K": K}
+        for name, qa_f, qw_f, g_f in (
+                ("fp32_scale", fb.fp8_quant_act_group128, fb.fp8_quant_weight_block128,
+                 fb.fp8_block_gemm),
+                ("ue8m0", fb.fp8_quant_act_group128_ue8m0, fb.fp8_quant_weight_block128_ue8m0,
+                 fb.fp8_block_gemm_ue8m0)):
+            y = g_f(*qa_f(xd), *qw_f(wd))
+            ys = y[r.to(dev)][:, c.to(dev)].double().cpu()
+            err = ys - exact
+            res[name] = {"rel_fro": float(err.norm() / exact.norm()),
+                         "max_abs_over_max_y": float(err.abs().max() / exact.abs().max())}
+        del xd, wd
+        out.append(res)
+    torch.cuda.empty_cache()
+    return out
 
 
 QUANT_SHAPES = (("quant_act", 8192, 0, 14336), ("quant_act", 8192, 0, 4096),
@@ -728,6 +782,7 @@ def run_ours(args, rank, world, local):
     if not args.no_sections:
         result["quantize"] = run_quantize(dev, stream, world)
         result["prefill"] = run_prefill(dev, stream, world)
+        result["accuracy"] = run_accuracy(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = OracleSample(seed=0)
         sample.run()   # first touch of the oracle's buffers, untimed

@@ -30,6 +30,9 @@ SIGNATURES = {
     "fp8_block_gemm": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_block_gemm_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_sparse24_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_quant_act_group128_ue8m0": (_I, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_quant_weight_block128_ue8m0": (_I, [_P, _I64, _I64, _P, _P, _P]),
+    "fp8_block_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
     "fp8bs_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -217,6 +220,52 @@ def fp8_sparse24_gemm(qa, sa, vals, meta, sw, y=None, workspace=None, stream=Non
     _check("fp8_sparse24_gemm",
            lib().fp8_sparse24_gemm(_ptr(qa), _ptr(sa), _ptr(vals), _ptr(meta), _ptr(sw), _ptr(y),
                                    M, N, K, _ptr(ws), ws_bytes, _stream(stream, qa)))
+    return y
+
+
+def fp8_quant_act_group128_ue8m0(x, qa=None, sa8=None, stream=None):
+    """x bf16 [M, K] -> (qa uint8 [M, K] E4M3 codes, sa8 uint8 [M, K/128] UE8M0 codes)."""
+    M, K = x.shape
+    _dev(x, torch.bfloat16, (M, K), "x")
+    qa = _empty((M, K), torch.uint8, x.device) if qa is None else qa
+    sa8 = _empty((M, K // 128), torch.uint8, x.device) if sa8 is None else sa8
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa8, torch.uint8, (M, K // 128), "sa8")
+    _check("fp8_quant_act_group128_ue8m0",
+           lib().fp8_quant_act_group128_ue8m0(_ptr(x), M, K, _ptr(qa), _ptr(sa8), _stream(stream, x)))
+    return qa, sa8
+
+
+def fp8_quant_weight_block128_ue8m0(w, qw=None, sw8=None, stream=None):
+    """w bf16 [N, K] -> (qw uint8 [N, K], sw8 uint8 [ceil(N/128), K/128] UE8M0 codes)."""
+    N, K = w.shape
+    _dev(w, torch.bfloat16, (N, K), "w")
+    NB = -(-N // 128)
+    qw = _empty((N, K), torch.uint8, w.device) if qw is None else qw
+    sw8 = _empty((NB, K // 128), torch.uint8, w.device) if sw8 is None else sw8
+    _dev(qw, torch.uint8, (N, K), "qw")
+    _dev(sw8, torch.uint8, (NB, K // 128), "sw8")
+    _check("fp8_quant_weight_block128_ue8m0",
+           lib().fp8_quant_weight_block128_ue8m0(_ptr(w), N, K, _ptr(qw), _ptr(sw8),
+                                                 _stream(stream, w)))
+    return qw, sw8
+
+
+def fp8_block_gemm_ue8m0(qa, sa8, qw, sw8, y=None, workspace=None, stream=None):
+    """Block-scaled FP8 GEMM with UE8M0 scales (the tensor cores' block scaling)."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    NB, KB = -(-N // 128), K // 128
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa8, torch.uint8, (M, KB), "sa8")
+    _dev(qw, torch.uint8, (N, K), "qw")
+    _dev(sw8, torch.uint8, (NB, KB), "sw8")
+    y = _empty((M, N), torch.bfloat16, qa.device) if y is None else y
+    _dev(y, torch.bfloat16, (M, N), "y")
+    ws, ws_bytes = _workspace(M, N, K, False, qa.device, workspace)
+    _check("fp8_block_gemm_ue8m0",
+           lib().fp8_block_gemm_ue8m0(_ptr(qa), _ptr(sa8), _ptr(qw), _ptr(sw8), _ptr(y), M, N, K,
+                                      _ptr(ws), ws_bytes, _stream(stream, qa)))
     return y
 
 

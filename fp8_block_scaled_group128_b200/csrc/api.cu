@@ -238,6 +238,49 @@ int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const u
                               static_cast<cudaStream_t>(stream));
 }
 
+int fp8_quant_act_group128_ue8m0(const void* x_bf16, int64_t M, int64_t K, void* qa_e4m3,
+                                 uint8_t* sa_ue8m0, void* stream) {
+  if (M < 0 || M > kMaxDim || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (M == 0) return FP8BS_OK;
+  if (!x_bf16 || !qa_e4m3 || !sa_ue8m0) return FP8BS_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(qa_e4m3) || !aligned16(sa_ue8m0)) return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_quant_act_group128_ue8m0(x_bf16, M, K, qa_e4m3, sa_ue8m0,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quant_weight_block128_ue8m0(const void* w_bf16, int64_t N, int64_t K, void* qw_e4m3,
+                                    uint8_t* sw_ue8m0, void* stream) {
+  if (N < 0 || N > 65535LL * 128 || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (N == 0) return FP8BS_OK;
+  if (!w_bf16 || !qw_e4m3 || !sw_ue8m0) return FP8BS_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(qw_e4m3) || !aligned16(sw_ue8m0)) return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_quant_weight_block128_ue8m0(w_bf16, N, K, qw_e4m3, sw_ue8m0,
+                                                      static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_block_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw,
+                         const uint8_t* sw_ue8m0, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (int st = check_gemm_args(M, N, K)) return st;
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa_ue8m0 || !qw || !sw_ue8m0 || !y_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned16(sa_ue8m0) || !aligned16(qw) || !aligned16(sw_ue8m0) ||
+      !aligned16(y_bf16))
+    return FP8BS_ERR_ALIGN;
+  (void)workspace;
+  (void)workspace_bytes;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_block_gemm_ue8m0(qa, sa_ue8m0, qw, sw_ue8m0, y_bf16, M, N, K, wait_limit(), err,
+                                 static_cast<cudaStream_t>(stream));
+}
+
 int fp8bs_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FP8BS_ERR_CUDA;
@@ -267,6 +310,6 @@ const char* fp8bs_status_string(int status) {
   }
 }
 
-int fp8bs_version(void) { return 100; }
+int fp8bs_version(void) { return 200; }
 
 }  // extern "C"

@@ -91,6 +91,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
+// mbar_wait by every lane of a warp with one verdict for all: the warp stays
+// converged even when the limit runs out for some lanes only.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));
+}
+
 // True in exactly one lane of the converged warp (elect.sync). A loop that
 // the whole warp runs, with only its issuing instruction under this
 // predicate, keeps its operands warp-uniform, which makes tcgen05 and TMA
@@ -302,6 +308,105 @@ __device__ __forceinline__ void mma_sp_f8f6f4_c(uint32_t d_tmem, uint64_t adesc,
       : "memory");
 }
 
+// Block-scaled MMA with UE8M0 scale factors read from TMEM:
+// D[tmem] (+)= (A * 2^sfa) * (B * 2^sfb)^T, kind::mxf8f6f4 (one scale per 32
+// elements along K of each row of A and of B; here the byte of each 32-bit
+// TMEM word selected by the descriptor's scale-factor ids, 0).
+__device__ __forceinline__ void mma_mxf8f6f4_bs(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t sfa_tmem,
+                                                uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes from shared memory into TMEM lanes [0, 32) of each
+// of the four lane quarters (the same data four times), 4 consecutive 32-bit
+// columns from `taddr` (the scale-factor layout of the block-scaled MMA).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// ------------------------------------------- CTA pairs (cta_group::2) --
+// A pair of CTAs (ranks 0 and 1 of a cluster of two) shares one MMA: rank 0
+// issues it, each CTA holds half of A (and of B) in its own shared memory at
+// the same offsets, and each CTA's TMEM holds its 128 rows of the result.
+
+// TMEM allocation for the pair: executed by the same warp of both CTAs with
+// the same destination slot.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// 3-D tiled bulk tensor load into this CTA's shared memory whose completion
+// (transaction bytes) is counted on the mbarrier at the shared::cluster
+// address `bar` of either CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// The block-scaled MMA of a CTA pair (issued by rank 0): M = 256 rows, 128 in
+// each CTA.
+__device__ __forceinline__ void mma_mxf8f6f4_bs_pair(uint32_t d_tmem, uint64_t adesc,
+                                                     uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// tmem_cp_32x128b_warpx4 for the pair: each CTA's shared memory (same
+// offset) into its own TMEM (same columns).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// One arrival on the mbarrier at the same offset in every CTA of `mask` once
+// all tcgen05 operations issued so far by this thread (for the pair) are
+// complete.
+__device__ __forceinline__ void mma_commit_pair_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+// Arrive (release at cluster scope) on an mbarrier of another CTA of the
+// cluster, at its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
 // Copy 128 rows x 16 bytes from shared memory (matrix descriptor) into TMEM:
 // row r lands in lane r, 4 consecutive 32-bit columns from `taddr`.
 __device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
@@ -412,6 +517,20 @@ __device__ __forceinline__ uint64_t noswizzle_kmajor_desc(uint32_t smem_addr, ui
 // a 2:4 sparse A (set by the caller), bits 0-1 select the metadata part (0).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: E4M3 x E4M3 ->
+// F32 (implicit), both operands K-major, UE8M0 scale factors (bit 23), N >> 3
+// in bits 17-22, M >> 4 in bits 24-28, scale-factor ids (bits 4-5 for B,
+// 29-30 for A) 0.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(int M, int N) {
+  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// The same descriptor reading byte `id` (0..3) of every scale-factor word of
+// A and of B.
+__host__ __device__ constexpr uint32_t idesc_with_sf_id(uint32_t idesc, uint32_t id) {
+  return idesc | (id << 29) | (id << 4);
 }
 
 // ----------------------------------------------------------------- cluster --

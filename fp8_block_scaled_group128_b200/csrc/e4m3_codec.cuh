@@ -160,6 +160,49 @@ __device__ __forceinline__ uint2 encode8(const uint4 v, const ScaleDivider& d) {
   return make_uint2(d.codes4(v.x, v.y), d.codes4(v.z, v.w));
 }
 
+// ----------------------------------------------------------- UE8M0 scales --
+// "Format d'échelle UE8M0": a scale stored as float8_e8m0fnu, a bare power of
+// two 2^(c - 127) (8 exponent bits, no sign, no mantissa). Chosen as the
+// smallest power of two s with 448 * s >= amax, so no element saturates.
+//
+// For amax = 1.f * 2^(E - 127) (E its biased exponent) and 448 = 1.75 * 2^8:
+// 448 * 2^e >= amax  <=>  e >= E - 135 + log2(1.f / 1.75), and since 1.f / 1.75
+// lies in (0.57, 1.15), the smallest such e is E - 135 when 1.f <= 1.75
+// (mantissa field <= 0x600000) and E - 134 otherwise; the code is e + 127,
+// clamped to 0..254 (zero and subnormal amax give code 0).
+__device__ __forceinline__ uint32_t ue8m0_code_of_amax(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int eb = static_cast<int>(b >> 23);
+  const int code = eb - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return eb == 0 ? 0u : static_cast<uint32_t>(min(max(code, 0), 254));
+}
+
+// 1 / s = 2^(127 - c) as an fp32 value (normal for c <= 253; 2^-127 for 254).
+__device__ __forceinline__ float ue8m0_inv_scale(uint32_t code) {
+  return code >= 254u ? __uint_as_float(0x00400000u) : __uint_as_float((254u - code) << 23);
+}
+
+// E4M3 codes of 8 bf16 values against a power-of-two scale: x * (1 / s) is
+// exact wherever it is a normal fp32 value and otherwise rounded once, so it
+// equals the IEEE quotient x / s; the product keeps the sign (also of zero)
+// and never exceeds 448 in magnitude (|x| <= amax <= 448 s).
+__device__ __forceinline__ uint32_t pow2_codes2(uint32_t w, uint64_t r2) {
+  float q0, q1;
+  asm("{\n\t.reg .b64 x, q;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mul.rn.f32x2 q, x, %4;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t}"
+      : "=f"(q0), "=f"(q1)
+      : "f"(__uint_as_float(w << 16)), "f"(__uint_as_float(w & 0xFFFF0000u)), "l"(r2));
+  return __nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ uint2 encode8_pow2(const uint4 v, float inv_scale) {
+  const uint64_t r2 = pack_f32x2(inv_scale, inv_scale);
+  return make_uint2(prmt(pow2_codes2(v.x, r2), pow2_codes2(v.y, r2), 0x5410u),
+                    prmt(pow2_codes2(v.z, r2), pow2_codes2(v.w, r2), 0x5410u));
+}
+
 // bf16x2 absmax word of 8 bf16 values (see absmax_to_float).
 __device__ __forceinline__ uint32_t absmax8(const uint4 v) {
   return bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w));

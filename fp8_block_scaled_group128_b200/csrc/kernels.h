@@ -15,6 +15,15 @@ cudaError_t launch_prune24_compress(const void* w, int64_t N, int64_t K, void* v
                                     uint8_t* meta, float* sw, void* w_pruned,
                                     cudaStream_t stream);
 
+// UE8M0 (power-of-two) scale variants: one code byte per group / block.
+cudaError_t launch_quant_act_group128_ue8m0(const void* x, int64_t M, int64_t K, void* qa,
+                                            uint8_t* sa8, cudaStream_t stream);
+cudaError_t launch_quant_weight_block128_ue8m0(const void* w, int64_t N, int64_t K, void* qw,
+                                               uint8_t* sw8, cudaStream_t stream);
+int launch_block_gemm_ue8m0(const void* qa, const uint8_t* sa8, const void* qw, const uint8_t* sw8,
+                            void* y, int64_t M, int64_t N, int64_t K, long long wait_limit,
+                            int* err, cudaStream_t stream);
+
 // Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
 // N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,

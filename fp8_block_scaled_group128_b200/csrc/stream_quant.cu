@@ -26,8 +26,9 @@ namespace fp8bs {
 
 namespace {
 
-// kPruneOut: 2:4 prune + compress that also writes the pruned bf16 weights.
-enum class QMode { kWeight, kPrune, kPruneOut };
+// kPruneOut: 2:4 prune + compress that also writes the pruned bf16 weights;
+// kWeightE8: weight blocks with UE8M0 (power-of-two) scales.
+enum class QMode { kWeight, kPrune, kPruneOut, kWeightE8 };
 
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
@@ -43,6 +44,7 @@ struct QArgs {
   uint8_t* q;              // codes [rows][K] (act / weight) or vals [N][K/2] (prune)
   uint8_t* meta;           // prune: [N][K/8]
   float* scale;            // act: [M][K/128]; weight / prune: [NB][K/128]
+  uint8_t* scale8;         // kWeightE8: UE8M0 codes [NB][K/128]
   __nv_bfloat16* pruned;   // prune: optional [N][K]
   long long wait_limit;
   int* err;
@@ -212,7 +214,19 @@ __global__ void __launch_bounds__(kQThreads, 2)
       }
     }
 
-    {
+    if constexpr (kMode == QMode::kWeightE8) {
+      const uint32_t code = ue8m0_code_of_amax(__uint_as_float(red[it % 3]));
+      if (t == 0) a.scale8[rb * KB + kb] = static_cast<uint8_t>(code);
+      const float inv = ue8m0_inv_scale(code);
+      const int64_t r0 = rb * 128 + (t >> 4);
+      const int rows_here = static_cast<int>(a.rows - r0 < 0 ? 0 : a.rows - r0);
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        if (i * (kQThreads / 16) >= rows_here) break;
+        const int64_t r = r0 + i * (kQThreads / 16);
+        reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8_pow2(v[i], inv);
+      }
+    } else {
       const float sc = scale_of_amax(__uint_as_float(red[it % 3]));
       if (t == 0) a.scale[rb * KB + kb] = sc;
       const ScaleDivider d(sc);
@@ -294,10 +308,11 @@ cudaError_t launch_stream(const void* x, int64_t rows, int64_t K, QArgs a, cudaS
 // barrier: for decode-sized inputs the kernel costs one load round trip.
 constexpr int kActThreads = 256;
 
-template <int kGroups>
+template <int kGroups, bool kE8 = false>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const __nv_bfloat16* __restrict__ x, int64_t groups,
-                     uint8_t* __restrict__ q, float* __restrict__ scale) {
+                     uint8_t* __restrict__ q, void* __restrict__ scale) {
+  // kE8: UE8M0 (power-of-two) scales, written as one code byte per group
   const int64_t teams = static_cast<int64_t>(gridDim.x) * (kActThreads / 16);
   const int64_t team = static_cast<int64_t>(blockIdx.x) * (kActThreads / 16) + (threadIdx.x >> 4);
   const int chunk = threadIdx.x & 15;
@@ -327,18 +342,29 @@ __global__ void __launch_bounds__(kActThreads)
     float m = absmax_to_float(absmax8(v[j]));
 #pragma unroll
     for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float sc = scale_of_amax(m);
-    if (g < groups) {
-      reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8(v[j], ScaleDivider(sc));
-      if (chunk == 0) scale[g] = sc;
+    if constexpr (kE8) {
+      const uint32_t code = ue8m0_code_of_amax(m);
+      if (g < groups) {
+        reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8_pow2(v[j], ue8m0_inv_scale(code));
+        if (chunk == 0) static_cast<uint8_t*>(scale)[g] = static_cast<uint8_t>(code);
+      }
+    } else {
+      const float sc = scale_of_amax(m);
+      if (g < groups) {
+        reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8(v[j], ScaleDivider(sc));
+        if (chunk == 0) static_cast<float*>(scale)[g] = sc;
+      }
     }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_quant_act_group128(const void* x, int64_t M, int64_t K, void* qa, float* sa,
-                                      cudaStream_t stream) {
+namespace {
+
+template <bool kE8>
+cudaError_t launch_act(const void* x, int64_t M, int64_t K, void* qa, void* sa,
+                       cudaStream_t stream) {
   DeviceInfo dev;
   if (current_device_info(&dev) != FP8BS_OK) return cudaErrorInvalidDevice;
   const int64_t groups = M * (K / 128);
@@ -359,8 +385,28 @@ cudaError_t launch_quant_act_group128(const void* x, int64_t M, int64_t K, void*
   cfg.numAttrs = 1;
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* qp = static_cast<uint8_t*>(qa);
-  return per == 4 ? cudaLaunchKernelEx(&cfg, act_quant_kernel<4>, xp, groups, qp, sa)
-                  : cudaLaunchKernelEx(&cfg, act_quant_kernel<1>, xp, groups, qp, sa);
+  return per == 4 ? cudaLaunchKernelEx(&cfg, act_quant_kernel<4, kE8>, xp, groups, qp, sa)
+                  : cudaLaunchKernelEx(&cfg, act_quant_kernel<1, kE8>, xp, groups, qp, sa);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act_group128(const void* x, int64_t M, int64_t K, void* qa, float* sa,
+                                      cudaStream_t stream) {
+  return launch_act<false>(x, M, K, qa, sa, stream);
+}
+
+cudaError_t launch_quant_act_group128_ue8m0(const void* x, int64_t M, int64_t K, void* qa,
+                                            uint8_t* sa8, cudaStream_t stream) {
+  return launch_act<true>(x, M, K, qa, sa8, stream);
+}
+
+cudaError_t launch_quant_weight_block128_ue8m0(const void* w, int64_t N, int64_t K, void* qw,
+                                               uint8_t* sw8, cudaStream_t stream) {
+  QArgs a{};
+  a.q = static_cast<uint8_t*>(qw);
+  a.scale8 = sw8;
+  return launch_stream<QMode::kWeightE8>(w, N, K, a, stream);
 }
 
 cudaError_t launch_quant_weight_block128(const void* w, int64_t N, int64_t K, void* qw, float* sw,

@@ -2,7 +2,8 @@
 
     python -m fp8_block_scaled_group128_b200.profile_case KIND M N K ITERS
 
-KIND is one of quant_act, quant_weight, prune24, dense_gemm, sparse_gemm.
+KIND is one of quant_act, quant_weight, prune24, dense_gemm, sparse_gemm,
+ue8m0_gemm.
 The inputs are the seeded synthetic llama tensors of that shape, prepared on
 the device by the library's own kernels before the ITERS launches of the
 kernel under test (select those with the profiler's kernel-name filter).
@@ -52,9 +53,9 @@ def main(argv):
     kind, M, N, K, iters = argv[0], int(argv[1]), int(argv[2]), int(argv[3]), int(argv[4])
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if kind in ("quant_weight", "prune24", "dense_gemm", "sparse_gemm"):
+    if kind in ("quant_weight", "prune24", "dense_gemm", "sparse_gemm", "ue8m0_gemm"):
         w = synth.weights("llama", N, K, seed=0).to(dev)
-    if kind in ("quant_act", "dense_gemm", "sparse_gemm"):
+    if kind in ("quant_act", "dense_gemm", "sparse_gemm", "ue8m0_gemm"):
         x = synth.activations("llama", max(M, 1), K, seed=0).to(dev)
 
     if kind == "quant_act":
@@ -80,6 +81,12 @@ def main(argv):
             vals, meta, sw, _ = fb.prune24_compress(w)
             fn = lambda: fb.fp8_sparse24_gemm(qa, sa, vals, meta, sw, y=y)  # noqa: E731
         del w
+    elif kind == "ue8m0_gemm":
+        qa, sa = fb.fp8_quant_act_group128_ue8m0(x)
+        qw, sw = fb.fp8_quant_weight_block128_ue8m0(w)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda: fb.fp8_block_gemm_ue8m0(qa, sa, qw, sw, y=y)  # noqa: E731
+        del w
     else:
         raise SystemExit(f"unknown kind {kind!r}")
     torch.cuda.synchronize()
@@ -91,8 +98,9 @@ def main(argv):
     torch.cuda.synchronize()
     if fb.get_device_error() != 0:
         raise SystemExit("device error")
-    print(f"{kind} M={M} N={N} K={K}: {e0.elapsed_time(e1) / iters * 1e3:.2f} us/launch "
-          f"over {iters} launches")
+    us = e0.elapsed_time(e1) / iters * 1e3
+    extra = f", {2.0 * M * N * K / (us * 1e-6) / 1e12:.1f} TFLOP/s" if kind.endswith("gemm") else ""
+    print(f"{kind} M={M} N={N} K={K}: {us:.2f} us/launch over {iters} launches{extra}")
 
 
 if __name__ == "__main__":

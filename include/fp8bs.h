@@ -154,6 +154,31 @@ int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const u
                       const float* sw, void* y_bf16, int64_t M, int64_t N, int64_t K,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * UE8M0 scale variant ("FP8 à granularité fine", section "Format d'échelle
+ * UE8M0": scales stored as float8_e8m0fnu, a bare power of two). A scale is
+ * kept as one code byte c standing for 2^(c - 127); it is the smallest power
+ * of two s with 448 * s >= amax (so no element saturates), codes clamped to
+ * 0..254, amax == 0 -> code 0. Elements are e4m3(x / s) as above (the quotient
+ * by a power of two is exact unless it underflows).
+ *
+ *   fp8_quant_act_group128_ue8m0:    x_bf16 [M][K] -> qa_e4m3 [M][K], sa_ue8m0 [M][K/128]
+ *   fp8_quant_weight_block128_ue8m0: w_bf16 [N][K] -> qw_e4m3 [N][K],
+ *                                    sw_ue8m0 [ceil(N/128)][K/128]
+ *   fp8_block_gemm_ue8m0: y = sum_kb 2^(sa - 127) 2^(sw - 127) (qa_kb . qw_kb^T),
+ *       fp32 accumulation, bf16 out (N a multiple of 8); the tensor cores apply
+ *       the scales themselves (block-scaled MMA), so there is no per-K-block
+ *       promotion. Workspace as fp8_block_gemm (none needed).
+ * Argument rules and errors as the fp32-scale entry points.
+ */
+int fp8_quant_act_group128_ue8m0(const void* x_bf16, int64_t M, int64_t K, void* qa_e4m3,
+                                 uint8_t* sa_ue8m0, void* stream);
+int fp8_quant_weight_block128_ue8m0(const void* w_bf16, int64_t N, int64_t K, void* qw_e4m3,
+                                    uint8_t* sw_ue8m0, void* stream);
+int fp8_block_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw,
+                         const uint8_t* sw_ue8m0, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Scratch bytes needed by the GEMMs for this shape (sparse != 0: the 2:4 GEMM). */
 size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse);
 

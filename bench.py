@@ -452,6 +452,7 @@ def run_prefill(dev, stream, world, reps=12):
         del fns, ins, qa, sa, wq, y, qy, sy
     wcache.clear()
     torch.cuda.empty_cache()
+    rows += run_grouped(dev, stream, world, peak, reps)
     agg = {k: v[0] / (v[1] * 1e-3) / 1e12 for k, v in tot.items()}
     return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
             "dense_achieved": round(agg["dense"], 1), "dense_frac": round(agg["dense"] / peak, 4),
@@ -462,6 +463,55 @@ def run_prefill(dev, stream, world, reps=12):
                     "1x128 quantization in the epilogue / after it (not in dense_achieved); inputs "
                     "rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
+
+
+def run_grouped(dev, stream, world, peak, reps=12):
+    """The grouped (mixture-of-experts) GEMMs on the DeepSeek-V3 expert
+    linears (gate+up N=4096 K=7168, down N=7168 K=2048): 8 experts, 4096
+    routed token rows with uneven loads, each expert's rows padded to 128
+    (synth.moe_layout), fp32 and UE8M0 scales. FLOPs count the routed rows
+    only (2 x routed x N x K)."""
+    from fp8_block_scaled_group128_b200 import binding as fb
+    from fp8_block_scaled_group128_b200 import synth
+    out = []
+    E, routed = synth.MOE_EXPERTS, synth.MOE_ROUTED_ROWS
+    for N, K in synth.MOE_LINEARS:
+        mi, _ = synth.moe_layout(E, routed, seed=3)
+        M = mi.numel()
+        with torch.cuda.stream(stream):
+            x = synth.activations("deepseek", M, K, seed=3).to(dev)
+            w = synth.expert_weights("deepseek", E, N, K, seed=3).to(dev)
+            mid = mi.to(dev)
+            NB, KB = -(-N // 128), K // 128
+            for fmt in ("fp32", "ue8m0"):
+                qw = torch.empty(E, N, K, dtype=torch.uint8, device=dev)
+                if fmt == "fp32":
+                    qa, sa = fb.fp8_quant_act_group128(x)
+                    sw = torch.empty(E, NB, KB, dtype=torch.float32, device=dev)
+                    for e in range(E):
+                        fb.fp8_quant_weight_block128(w[e], qw=qw[e], sw=sw[e])
+                    gemm = fb.fp8_grouped_gemm
+                else:
+                    qa, sa = fb.fp8_quant_act_group128_ue8m0(x)
+                    sw = torch.empty(E, NB, KB, dtype=torch.uint8, device=dev)
+                    for e in range(E):
+                        fb.fp8_quant_weight_block128_ue8m0(w[e], qw=qw[e], sw8=sw[e])
+                    gemm = fb.fp8_grouped_gemm_ue8m0
+                y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                n_cp = copies_beyond_l2(M * K + E * N * K, cap=4)
+                ins = [(qa, sa, qw, sw)] + [(qa.clone(), sa.clone(), qw.clone(), sw.clone())
+                                            for _ in range(n_cp - 1)]
+                fns = [lambda i=i: gemm(*i, mid, y=y) for i in ins]
+                ms = _time_graph(fns, stream, world, reps)
+                tf = 2.0 * routed * N * K / (ms * 1e-3) / 1e12
+                out.append({"gemm": f"grouped_{fmt}", "experts": E, "M_routed": routed,
+                            "M_padded": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
+                            "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
+                            "input_copies": n_cp})
+                del fns, ins, qa, sa, qw, sw, y
+            del x, w
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_accuracy(dev):

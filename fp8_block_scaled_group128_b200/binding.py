@@ -33,6 +33,8 @@ SIGNATURES = {
     "fp8_quant_act_group128_ue8m0": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_quant_weight_block128_ue8m0": (_I, [_P, _I64, _I64, _P, _P, _P]),
     "fp8_block_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_grouped_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_grouped_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
     "fp8bs_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -267,6 +269,33 @@ def fp8_block_gemm_ue8m0(qa, sa8, qw, sw8, y=None, workspace=None, stream=None):
            lib().fp8_block_gemm_ue8m0(_ptr(qa), _ptr(sa8), _ptr(qw), _ptr(sw8), _ptr(y), M, N, K,
                                       _ptr(ws), ws_bytes, _stream(stream, qa)))
     return y
+
+
+def _grouped(name, qa, sa, qw, sw, m_indices, y, scale_dtype, stream):
+    M, K = qa.shape
+    E, N, _ = qw.shape
+    NB, KB = -(-N // 128), K // 128
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa, scale_dtype, (M, KB), "sa")
+    _dev(qw, torch.uint8, (E, N, K), "qw")
+    _dev(sw, scale_dtype, (E, NB, KB), "sw")
+    _dev(m_indices, torch.int32, (M,), "m_indices")
+    y = _empty((M, N), torch.bfloat16, qa.device) if y is None else y
+    _dev(y, torch.bfloat16, (M, N), "y")
+    _check(name, getattr(lib(), name)(_ptr(qa), _ptr(sa), _ptr(qw), _ptr(sw), _ptr(m_indices),
+                                      _ptr(y), M, N, K, E, None, 0, _stream(stream, qa)))
+    return y
+
+
+def fp8_grouped_gemm(qa, sa, qw, sw, m_indices, y=None, stream=None):
+    """Mixture-of-experts block-scaled GEMM (fp32 scales): row m of qa uses the
+    weights qw[m_indices[m]] ([E, N, K]); each 128-row tile holds one expert."""
+    return _grouped("fp8_grouped_gemm", qa, sa, qw, sw, m_indices, y, torch.float32, stream)
+
+
+def fp8_grouped_gemm_ue8m0(qa, sa8, qw, sw8, m_indices, y=None, stream=None):
+    """The grouped GEMM with UE8M0 scale codes."""
+    return _grouped("fp8_grouped_gemm_ue8m0", qa, sa8, qw, sw8, m_indices, y, torch.uint8, stream)
 
 
 def get_device_error(stream=None, device=None):

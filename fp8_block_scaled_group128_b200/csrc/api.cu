@@ -22,6 +22,10 @@ std::atomic<long long> g_wait_limit{kDefaultWaitCycles};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Scale arrays (fp32 scales or UE8M0 codes) and expert indices are read with
+// loads of at most 4 bytes.
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
 int check_k(int64_t K) { return (K <= 0 || K % 128 != 0) ? FP8BS_ERR_SHAPE : FP8BS_OK; }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP8BS_OK : FP8BS_ERR_CUDA; }
@@ -136,7 +140,7 @@ int fp8_quant_act_group128(const void* x_bf16, int64_t M, int64_t K, void* qa_e4
   if (int st = check_k(K)) return st;
   if (M == 0) return FP8BS_OK;
   if (!x_bf16 || !qa_e4m3 || !sa) return FP8BS_ERR_NULL;
-  if (!aligned16(x_bf16) || !aligned16(qa_e4m3) || !aligned16(sa)) return FP8BS_ERR_ALIGN;
+  if (!aligned16(x_bf16) || !aligned16(qa_e4m3) || !aligned4(sa)) return FP8BS_ERR_ALIGN;
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
   return from_cuda(launch_quant_act_group128(x_bf16, M, K, qa_e4m3, sa,
@@ -149,7 +153,7 @@ int fp8_quant_weight_block128(const void* w_bf16, int64_t N, int64_t K, void* qw
   if (int st = check_k(K)) return st;
   if (N == 0) return FP8BS_OK;
   if (!w_bf16 || !qw_e4m3 || !sw) return FP8BS_ERR_NULL;
-  if (!aligned16(w_bf16) || !aligned16(qw_e4m3) || !aligned16(sw)) return FP8BS_ERR_ALIGN;
+  if (!aligned16(w_bf16) || !aligned16(qw_e4m3) || !aligned4(sw)) return FP8BS_ERR_ALIGN;
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
   return from_cuda(launch_quant_weight_block128(w_bf16, N, K, qw_e4m3, sw,
@@ -162,7 +166,7 @@ int prune24_compress(const void* w_bf16, int64_t N, int64_t K, void* vals_e4m3, 
   if (int st = check_k(K)) return st;
   if (N == 0) return FP8BS_OK;
   if (!w_bf16 || !vals_e4m3 || !meta || !sw) return FP8BS_ERR_NULL;
-  if (!aligned16(w_bf16) || !aligned16(vals_e4m3) || !aligned16(meta) || !aligned16(sw) ||
+  if (!aligned16(w_bf16) || !aligned16(vals_e4m3) || !aligned16(meta) || !aligned4(sw) ||
       (w_pruned_bf16 && !aligned16(w_pruned_bf16)))
     return FP8BS_ERR_ALIGN;
   DeviceInfo dev;
@@ -192,7 +196,7 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
   if (int st = check_gemm_args(M, N, K)) return st;
   if (M == 0 || N == 0) return FP8BS_OK;
   if (!qa || !sa || !qw || !sw || !y_bf16) return FP8BS_ERR_NULL;
-  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) || !aligned16(y_bf16))
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw) || !aligned4(sw) || !aligned16(y_bf16))
     return FP8BS_ERR_ALIGN;
   if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 0)) return FP8BS_ERR_WORKSPACE;
   (void)workspace;
@@ -210,8 +214,8 @@ int fp8_block_gemm_quant(const void* qa, const float* sa, const void* qw, const 
   if (M == 0 || N == 0) return FP8BS_OK;
   if (!qa || !sa || !qw || !sw || !qy_e4m3 || !sy) return FP8BS_ERR_NULL;
   if (M <= 256 && !y_bf16) return FP8BS_ERR_NULL;  // decode-sized M quantizes the stored Y
-  if (!aligned16(qa) || !aligned16(sa) || !aligned16(qw) || !aligned16(sw) ||
-      (y_bf16 && !aligned16(y_bf16)) || !aligned16(qy_e4m3) || !aligned16(sy))
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw) || !aligned4(sw) ||
+      (y_bf16 && !aligned16(y_bf16)) || !aligned16(qy_e4m3) || !aligned4(sy))
     return FP8BS_ERR_ALIGN;
   if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 0)) return FP8BS_ERR_WORKSPACE;
   (void)workspace;
@@ -227,8 +231,8 @@ int fp8_sparse24_gemm(const void* qa, const float* sa, const void* vals, const u
   if (int st = check_gemm_args(M, N, K)) return st;
   if (M == 0 || N == 0) return FP8BS_OK;
   if (!qa || !sa || !vals || !meta || !sw || !y_bf16) return FP8BS_ERR_NULL;
-  if (!aligned16(qa) || !aligned16(sa) || !aligned16(vals) || !aligned16(meta) ||
-      !aligned16(sw) || !aligned16(y_bf16))
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(vals) || !aligned16(meta) ||
+      !aligned4(sw) || !aligned16(y_bf16))
     return FP8BS_ERR_ALIGN;
   if (workspace_bytes < fp8bs_gemm_workspace_bytes(M, N, K, 1)) return FP8BS_ERR_WORKSPACE;
   (void)workspace;
@@ -244,7 +248,7 @@ int fp8_quant_act_group128_ue8m0(const void* x_bf16, int64_t M, int64_t K, void*
   if (int st = check_k(K)) return st;
   if (M == 0) return FP8BS_OK;
   if (!x_bf16 || !qa_e4m3 || !sa_ue8m0) return FP8BS_ERR_NULL;
-  if (!aligned16(x_bf16) || !aligned16(qa_e4m3) || !aligned16(sa_ue8m0)) return FP8BS_ERR_ALIGN;
+  if (!aligned16(x_bf16) || !aligned16(qa_e4m3)) return FP8BS_ERR_ALIGN;
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
   return from_cuda(launch_quant_act_group128_ue8m0(x_bf16, M, K, qa_e4m3, sa_ue8m0,
@@ -257,7 +261,7 @@ int fp8_quant_weight_block128_ue8m0(const void* w_bf16, int64_t N, int64_t K, vo
   if (int st = check_k(K)) return st;
   if (N == 0) return FP8BS_OK;
   if (!w_bf16 || !qw_e4m3 || !sw_ue8m0) return FP8BS_ERR_NULL;
-  if (!aligned16(w_bf16) || !aligned16(qw_e4m3) || !aligned16(sw_ue8m0)) return FP8BS_ERR_ALIGN;
+  if (!aligned16(w_bf16) || !aligned16(qw_e4m3)) return FP8BS_ERR_ALIGN;
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;
   return from_cuda(launch_quant_weight_block128_ue8m0(w_bf16, N, K, qw_e4m3, sw_ue8m0,
@@ -270,7 +274,7 @@ int fp8_block_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw
   if (int st = check_gemm_args(M, N, K)) return st;
   if (M == 0 || N == 0) return FP8BS_OK;
   if (!qa || !sa_ue8m0 || !qw || !sw_ue8m0 || !y_bf16) return FP8BS_ERR_NULL;
-  if (!aligned16(qa) || !aligned16(sa_ue8m0) || !aligned16(qw) || !aligned16(sw_ue8m0) ||
+  if (!aligned16(qa) || !aligned16(qw) ||
       !aligned16(y_bf16))
     return FP8BS_ERR_ALIGN;
   (void)workspace;
@@ -279,6 +283,47 @@ int fp8_block_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw
   if (err == nullptr) return FP8BS_ERR_CUDA;
   return launch_block_gemm_ue8m0(qa, sa_ue8m0, qw, sw_ue8m0, y_bf16, M, N, K, wait_limit(), err,
                                  static_cast<cudaStream_t>(stream));
+}
+
+static int check_grouped_args(int64_t M, int64_t N, int64_t K, int64_t E) {
+  if (int st = check_gemm_args(M, N, K)) return st;
+  if (E < 1 || E > kMaxDim || (N > 0 && E > kMaxDim / N)) return FP8BS_ERR_SHAPE;
+  return FP8BS_OK;
+}
+
+int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const float* sw,
+                     const int32_t* m_indices, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                     int64_t E, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int st = check_grouped_args(M, N, K, E)) return st;
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa || !qw || !sw || !m_indices || !y_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw) || !aligned4(sw) ||
+      !aligned4(m_indices) || !aligned16(y_bf16))
+    return FP8BS_ERR_ALIGN;
+  (void)workspace;
+  (void)workspace_bytes;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_block_gemm_grouped(qa, sa, qw, sw, m_indices, y_bf16, M, N, K, E, wait_limit(),
+                                   err, static_cast<cudaStream_t>(stream));
+}
+
+int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw,
+                           const uint8_t* sw_ue8m0, const int32_t* m_indices, void* y_bf16,
+                           int64_t M, int64_t N, int64_t K, int64_t E, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (int st = check_grouped_args(M, N, K, E)) return st;
+  if (M == 0 || N == 0) return FP8BS_OK;
+  if (!qa || !sa_ue8m0 || !qw || !sw_ue8m0 || !m_indices || !y_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned16(qw) ||
+      !aligned4(m_indices) || !aligned16(y_bf16))
+    return FP8BS_ERR_ALIGN;
+  (void)workspace;
+  (void)workspace_bytes;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_block_gemm_grouped_ue8m0(qa, sa_ue8m0, qw, sw_ue8m0, m_indices, y_bf16, M, N, K,
+                                         E, wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
 int fp8bs_get_device_error(void* stream) {
@@ -301,7 +346,7 @@ const char* fp8bs_status_string(int status) {
     case FP8BS_OK: return "ok";
     case FP8BS_ERR_NULL: return "a required pointer is NULL";
     case FP8BS_ERR_SHAPE: return "invalid shape (K must be a positive multiple of 128; N a multiple of 8 for GEMMs)";
-    case FP8BS_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case FP8BS_ERR_ALIGN: return "a pointer is not aligned (16 bytes for matrices, 4 for fp32 scales and indices)";
     case FP8BS_ERR_WORKSPACE: return "workspace too small";
     case FP8BS_ERR_CUDA: return "CUDA call failed";
     case FP8BS_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";

@@ -72,4 +72,37 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
 }
 
+int launch_block_gemm_grouped(const void* qa, const float* sa, const void* qw, const float* sw,
+                              const int* m_indices, void* y, int64_t M, int64_t N, int64_t K,
+                              int64_t E, long long wait_limit, int* err, cudaStream_t stream) {
+  // The prefill-order kernel for every M: tiles of 128 token rows (one
+  // expert each) x 256 rows of that expert's weights.
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  GemmArgs a{};
+  a.sa = sa;
+  a.sw = sw;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.KB = static_cast<int>(K / 128);
+  a.NB = static_cast<int>((N + 127) / 128);
+  a.wait_limit = wait_limit;
+  a.err = err;
+  a.m_indices = m_indices;
+  a.E = static_cast<int>(E);
+  constexpr int BN = 256;
+  a.row_tiles = static_cast<int>((M + 127) / 128);
+  a.col_tiles = static_cast<int>((N + BN - 1) / BN);
+  a.splits = 1;
+  const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
+  if (tiles > 0x7FFFFFFF) return FP8BS_ERR_SHAPE;
+  const int grid_y = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  const uint64_t KB = static_cast<uint64_t>(K / 128);
+  alignas(64) CUtensorMap ta, tb;
+  if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, 128, 1, kSwizzle128B)) return st;
+  if (int st = encode_tmap_kblocks(&tb, qw, 128, E * N, KB, K, BN, 1, kSwizzle128B)) return st;
+  return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
+}
+
 }  // namespace fp8bs

@@ -72,7 +72,20 @@ struct GemmArgs {
   int* err;             // device error word
   uint8_t* qy;          // kQOut: Y quantized in 1x128 groups along N, [M][N] E4M3
   float* sy;            // kQOut: their scales, [M][N/128]
+  // Grouped (mixture-of-experts) GEMM, prefill order only: the expert of
+  // every token row ([M], null = one weight matrix); weights [E][N][K] and
+  // scales [E][NB][KB]. Every 128-row tile takes the expert of its first row
+  // (indices outside [0, E) count as expert 0).
+  const int* m_indices;
+  int E;
 };
+
+// Expert of row tile `rt` of a grouped GEMM (0 when not grouped).
+__device__ __forceinline__ int tile_expert(const GemmArgs& a, int rt) {
+  if (a.m_indices == nullptr) return 0;
+  const int e = __ldg(a.m_indices + static_cast<int64_t>(rt) * 128);
+  return (e < 0 || e >= a.E) ? 0 : e;
+}
 
 // Split-K over a cluster of S CTAs: rank q reduces weight rows
 // [recv_lo(q, S), recv_lo(q + 1, S)) of the 128-row tile (multiples of 4).
@@ -296,6 +309,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     for (int tile = blockIdx.y; tile < num_tiles && !*abort_flag; tile += gridDim.y) {
       int rt, ct;
       tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
+      // weight rows of this tile (of its expert, for a grouped GEMM)
+      const int brow = ct * BN + (kSwap ? 0 : tile_expert(args, rt) * args.N);
       for (int kb = kb0; kb < kb1; kb += kKS) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, limit)) {
           record_device_error(args.err, FP8BS_ERR_DEVICE_TIMEOUT);
@@ -309,7 +324,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           tma_load_3d(sm_a + stage * C::kABytes, &tmap_a, &full[stage], 0, rt * 128, kb);
           if constexpr (kSparse)
             tma_load_3d(sm_e + stage * C::kEStage, &tmap_e, &full[stage], 0, rt * 128, kb);
-          tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, ct * BN, kb);
+          tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, brow, kb);
         }
         __syncwarp();
         ++issued;
@@ -452,6 +467,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     // raster costs three integer divisions, a long dependency chain that
     // would otherwise stall every group boundary)
     int grt = 0, gct = 0;
+    int64_t gsw = 0;   // prefill: offset of the staged tile's expert in sW
     // Thread e stages table entries (K-block sg of the group, slot s0 + i *
     // kSlotStep) for i < kPer: the same K-block for every i. In decode order
     // its first token and the scale pointers at K-block sg are fixed per
@@ -465,6 +481,8 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
     const float* w0 = args.sw;
     auto tile_bases = [&]() {
       tile_coords(g_tile, args.row_tiles, args.col_tiles, grt, gct);
+      if constexpr (!kSwap)
+        gsw = static_cast<int64_t>(tile_expert(args, grt)) * args.NB * args.KB;
       if constexpr (kSwap) {
         first = gct * BN + s0;
         nb0 = grt;
@@ -496,7 +514,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           const int kb = g_kb + sg;
           if (kb_ok && m < args.M && nb < args.NB) {
             va = args.sa[m * KB + kb];
-            vw = args.sw[nb * KB + kb];
+            vw = args.sw[gsw + nb * KB + kb];
           }
         }
         pre_a[i] = va;

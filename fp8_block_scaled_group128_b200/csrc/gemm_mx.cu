@@ -99,7 +99,20 @@ struct MxArgs {
   int row_tiles, col_tiles;   // tiles of kP * 128 token rows and 256 weight rows
   long long wait_limit;
   int* err;
+  // Grouped (mixture-of-experts) GEMM, kP = 1: the expert of every token row
+  // ([M], null = one weight matrix); weights [E][N][K], codes [E][NB][KB].
+  // Every 128-row tile takes the expert of its first row (indices outside
+  // [0, E) count as expert 0).
+  const int* m_indices;
+  int E;
+  bool words_ok;   // both code arrays 4-byte aligned: a group's codes load as one word
 };
+
+__device__ __forceinline__ int mx_tile_expert(const MxArgs& a, int rt) {
+  if (a.m_indices == nullptr) return 0;
+  const int e = __ldg(a.m_indices + static_cast<int64_t>(rt) * kBM);
+  return (e < 0 || e >= a.E) ? 0 : e;
+}
 
 template <int kP>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -186,6 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = unit; tile < num_tiles && !aborted(); tile += units) {
       int rt, ct;
       gemm_detail::tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
+      // weight rows of this CTA's half of the tile (of its expert, if grouped)
+      const int brow = ct * kBN + rank * C::kBNc + mx_tile_expert(args, rt) * args.N;
+      const int arow = (rt * kP + rank) * kBM;
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait_warp(&empty[stage], phase ^ 1u, limit)) {
@@ -197,8 +213,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) {
           uint8_t* da = sm_a + stage * kABytes;
           uint8_t* db = sm_b + stage * C::kBBytes;
-          const int arow = (rt * kP + rank) * kBM;
-          const int brow = ct * kBN + rank * C::kBNc;
           if constexpr (kP == 2) {
             if (leader) mbar_arrive_expect_tx(&full_tma[stage], kP * (kABytes + C::kBBytes));
             const uint32_t bar = leader_bar(&full_tma[stage]);
@@ -373,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t a[4];
       uint32_t b[2];
     };
-    const bool kb_aligned = KB % kGroupK == 0;   // groups are whole, 4-byte aligned words
+    // groups are whole, 4-byte aligned words
+    const bool kb_aligned = KB % kGroupK == 0 && args.words_ok;
     auto word_of = [&](const uint8_t* row_codes, int kg) -> uint32_t {
       if (kb_aligned) return *reinterpret_cast<const uint32_t*>(row_codes + kg);
       uint32_t w = 0;
@@ -389,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int rt, ct;
       gemm_detail::tile_coords(tile, args.row_tiles, args.col_tiles, rt, ct);
       const int nb0 = ct * (kBN / 128);
+      const uint8_t* sw8 = args.sw8 + static_cast<int64_t>(mx_tile_expert(args, rt)) * args.NB * KB;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int row = (rt * kP + rank) * kBM + lane + 32 * j;
@@ -396,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        if (nb0 + h < args.NB) c.b[h] = word_of(args.sw8 + static_cast<int64_t>(nb0 + h) * KB, kg);
+        if (nb0 + h < args.NB) c.b[h] = word_of(sw8 + static_cast<int64_t>(nb0 + h) * KB, kg);
     };
     const uint32_t sf_full_leader0 = leader_bar(&sf_full[0]);
     int q = 0;
@@ -498,6 +514,7 @@ template <int kP>
 int launch_mx(const void* qa, const void* qw, MxArgs a, int64_t M, int64_t N, int64_t K,
               const DeviceInfo& dev, cudaStream_t stream) {
   using C = MxCfg<kP>;
+  a.words_ok = ((reinterpret_cast<uintptr_t>(a.sa8) | reinterpret_cast<uintptr_t>(a.sw8)) & 3u) == 0;
   a.row_tiles = static_cast<int>((M + kP * kBM - 1) / (kP * kBM));
   a.col_tiles = static_cast<int>((N + kBN - 1) / kBN);
   const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
@@ -505,7 +522,9 @@ int launch_mx(const void* qa, const void* qw, MxArgs a, int64_t M, int64_t N, in
   const uint64_t KB = static_cast<uint64_t>(K / 128);
   alignas(64) CUtensorMap ta, tb;
   if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, kBM, 1, kSwizzle128B)) return st;
-  if (int st = encode_tmap_kblocks(&tb, qw, 128, N, KB, K, C::kBNc, 1, kSwizzle128B)) return st;
+  const uint64_t b_rows = static_cast<uint64_t>(N) * (a.m_indices != nullptr ? a.E : 1);
+  if (int st = encode_tmap_kblocks(&tb, qw, 128, b_rows, KB, K, C::kBNc, 1, kSwizzle128B))
+    return st;
   auto kern = mx_gemm_kernel<kP>;
   static std::once_flag flags[64];
   cudaError_t attr_err = cudaSuccess;
@@ -564,6 +583,29 @@ int launch_block_gemm_ue8m0(const void* qa, const uint8_t* sa8, const void* qw, 
   a.err = err;
   // a pair needs two 128-row halves to fill its M = 256 MMA
   if (M > kBM) return launch_mx<2>(qa, qw, a, M, N, K, dev, stream);
+  return launch_mx<1>(qa, qw, a, M, N, K, dev, stream);
+}
+
+int launch_block_gemm_grouped_ue8m0(const void* qa, const uint8_t* sa8, const void* qw,
+                                    const uint8_t* sw8, const int* m_indices, void* y, int64_t M,
+                                    int64_t N, int64_t K, int64_t E, long long wait_limit, int* err,
+                                    cudaStream_t stream) {
+  using namespace mx_detail;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  MxArgs a{};
+  a.sa8 = sa8;
+  a.sw8 = sw8;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.KB = static_cast<int>(K / 128);
+  a.NB = static_cast<int>((N + 127) / 128);
+  a.wait_limit = wait_limit;
+  a.err = err;
+  a.m_indices = m_indices;
+  a.E = static_cast<int>(E);
+  // single-CTA tiles of 128 token rows: one expert per tile
   return launch_mx<1>(qa, qw, a, M, N, K, dev, stream);
 }
 

@@ -24,6 +24,17 @@ int launch_block_gemm_ue8m0(const void* qa, const uint8_t* sa8, const void* qw, 
                             void* y, int64_t M, int64_t N, int64_t K, long long wait_limit,
                             int* err, cudaStream_t stream);
 
+// Grouped (mixture-of-experts) block-scaled GEMMs: token row m uses the
+// weights of expert m_indices[m] (weights [E][N][K]); every 128-row tile
+// belongs to one expert. Return FP8BS_* status.
+int launch_block_gemm_grouped(const void* qa, const float* sa, const void* qw, const float* sw,
+                              const int* m_indices, void* y, int64_t M, int64_t N, int64_t K,
+                              int64_t E, long long wait_limit, int* err, cudaStream_t stream);
+int launch_block_gemm_grouped_ue8m0(const void* qa, const uint8_t* sa8, const void* qw,
+                                    const uint8_t* sw8, const int* m_indices, void* y, int64_t M,
+                                    int64_t N, int64_t K, int64_t E, long long wait_limit, int* err,
+                                    cudaStream_t stream);
+
 // Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
 // N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,

@@ -32,6 +32,12 @@ PREFILL_M = (2048, 8192)
 # (N, K) of the DeepSeek-V3 block-scaled linears.
 DEEPSEEK_V3_LINEARS = ((2112, 7168), (24576, 7168), (7168, 7168), (4096, 7168), (7168, 2048))
 DEEPSEEK_M = (64, 4096)
+# Mixture-of-experts linears of DeepSeek-V3 (an expert's gate+up and down
+# projections, intermediate size 2048): (N, K).
+MOE_LINEARS = ((4096, 7168), (7168, 2048))
+MOE_EXPERTS = 8
+MOE_ROUTED_ROWS = 4096
+MOE_ALIGN = 128
 # 2:4 sparse weights and token counts.
 SPARSE_LINEARS = ((14336, 4096), (4096, 14336))
 SPARSE_M = (16, 4096)
@@ -87,3 +93,30 @@ def uniform_bf16(shape, lo, hi, seed=0, tag="u"):
     """bf16 values uniform in [lo, hi) (edge-case tests)."""
     g = _gen(seed, tag, *shape)
     return (torch.rand(*shape, generator=g) * (hi - lo) + lo).to(torch.bfloat16)
+
+
+def moe_layout(experts, routed_rows, seed=0, align=128):
+    """Seeded expert assignment of `routed_rows` token rows in the contiguous
+    grouped layout: each expert's rows are consecutive, its segment is padded
+    with rows of index -1 to a multiple of `align`, experts in order. The
+    per-expert loads are a multinomial draw over Dirichlet(1) weights (uneven
+    loads, as routers produce). Returns (m_indices int32 [rows], counts)."""
+    g = _gen(seed, "moe", experts, routed_rows, align)
+    # Dirichlet(1) weights as normalised exponentials (drawn with the seeded
+    # generator, so the layout is reproducible)
+    e = -torch.log(torch.rand(experts, generator=g, dtype=torch.float64).clamp_min(1e-300))
+    p = e / e.sum()
+    counts = torch.multinomial(p, routed_rows, replacement=True, generator=g).bincount(
+        minlength=experts)
+    parts = []
+    for i, c in enumerate(counts.tolist()):
+        pad = (-c) % align
+        parts.append(torch.full((c,), i, dtype=torch.int32))
+        parts.append(torch.full((pad,), -1, dtype=torch.int32))
+    return torch.cat(parts), counts
+
+
+def expert_weights(kind, experts, N, K, seed=0):
+    """bf16 weights [E, N, K] of `experts` experts (each drawn like
+    weights(kind, N, K) with its own seed)."""
+    return torch.stack([weights(kind, N, K, seed=seed * 1000 + i) for i in range(experts)])

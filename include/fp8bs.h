@@ -33,7 +33,9 @@
  *   - All matrices are dense row-major, with no leading-dimension argument.
  *   - K must be a positive multiple of 128. M == 0 or N == 0 is a no-op that
  *     returns FP8BS_OK.
- *   - Every data pointer must be 16-byte aligned.
+ *   - Every matrix pointer (activations, weights, codes, metadata, outputs)
+ *     must be 16-byte aligned; fp32 scale arrays and expert indices need
+ *     4-byte alignment; UE8M0 scale-code arrays (bytes) need none.
  *   - Arguments are validated before anything is launched; on an error
  *     nothing is written and a nonzero FP8BS_ERR_* code is returned.
  *   - A launch failure returns FP8BS_ERR_CUDA. A kernel that gave up a bounded
@@ -55,7 +57,7 @@ typedef enum {
   FP8BS_OK = 0,
   FP8BS_ERR_NULL = 1,           /* a required pointer is NULL */
   FP8BS_ERR_SHAPE = 2,          /* K % 128 != 0, K <= 0, M/N < 0, or a size too large */
-  FP8BS_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+  FP8BS_ERR_ALIGN = 3,          /* a pointer is not aligned (16 bytes; 4 for scales / indices) */
   FP8BS_ERR_WORKSPACE = 4,      /* workspace smaller than fp8bs_gemm_workspace_bytes() */
   FP8BS_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
   FP8BS_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up a bounded wait */
@@ -178,6 +180,35 @@ int fp8_quant_weight_block128_ue8m0(const void* w_bf16, int64_t N, int64_t K, vo
 int fp8_block_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw,
                          const uint8_t* sw_ue8m0, void* y_bf16, int64_t M, int64_t N, int64_t K,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Grouped (mixture-of-experts) block-scaled GEMMs ("FP8 à granularité fine",
+ * section "Chemin rapide de DeepGEMM": the experts' products run through
+ * grouped kernels; with UE8M0 scales on SM100 per section "Format d'échelle
+ * UE8M0", with fp32 scales as a grouped matmul). The token rows are grouped
+ * by expert in one matrix (the contiguous layout):
+ *
+ *   y[m][n] = sum_kb sa[m][kb] * sw[e][n/128][kb] * sum_{k in kb} qa[m][k] qw[e][n][k],
+ *             e = m_indices[m]
+ *
+ *   qa [M][K] E4M3, sa [M][K/128] (fp32, or UE8M0 codes for the _ue8m0 form).
+ *   qw [E][N][K] E4M3, sw [E][ceil(N/128)][K/128] (fp32, or UE8M0 codes).
+ *   m_indices [M] int32, device memory: the expert of each row, or -1 for a
+ *       padding row. Every aligned group of 128 rows (rows 128t .. 128t+127)
+ *       must hold rows of a single expert plus padding rows: each expert's
+ *       rows start at a multiple of 128. The expert of a tile is read from its
+ *       first row; an index outside [0, E) there counts as expert 0.
+ *   y_bf16 [M][N]: rows of real tokens are written; padding rows receive
+ *       values with no defined meaning.
+ * N a multiple of 8, K of 128, E >= 1. Same errors as fp8_block_gemm.
+ */
+int fp8_grouped_gemm(const void* qa, const float* sa, const void* qw, const float* sw,
+                     const int32_t* m_indices, void* y_bf16, int64_t M, int64_t N, int64_t K,
+                     int64_t E, void* workspace, size_t workspace_bytes, void* stream);
+int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* qw,
+                           const uint8_t* sw_ue8m0, const int32_t* m_indices, void* y_bf16,
+                           int64_t M, int64_t N, int64_t K, int64_t E, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /* Scratch bytes needed by the GEMMs for this shape (sparse != 0: the 2:4 GEMM). */
 size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse);

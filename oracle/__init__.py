@@ -29,6 +29,8 @@ from .fp8_oracle_cpp import (  # noqa: F401
     gemm_abs_sum,
     gemm_error_bound,
     gemm_error_bound_ue8m0,
+    grouped_gemm,
+    grouped_gemm_ue8m0,
     prune24_compress,
     quant_act_group128,
     quant_act_group128_ue8m0,

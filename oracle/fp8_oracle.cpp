@@ -416,6 +416,41 @@ void orc_sparse24_gemm(const uint8_t* qa, const float* sa, int64_t M, const uint
   });
 }
 
+// The grouped (mixture-of-experts) GEMM: row m of the tokens is multiplied by
+// the weights of its expert e = m_indices[m] (weights [E][N][K], scales
+// [E][ceil(N/128)][K/128]) with the block-scaled formula above; rows with
+// e outside [0, E) (padding) get NaN, i.e. no defined result.
+void orc_grouped_gemm(const uint8_t* qa, const float* sa, int64_t M, const uint8_t* qw,
+                      const float* sw, const int32_t* m_indices, int64_t E, int64_t N, int64_t K,
+                      double* y) {
+  const int64_t KB = K / kGroup, NB = (N + kGroup - 1) / kGroup;
+  double table[256];
+  for (int c = 0; c < 256; ++c) table[c] = e4m3_value(static_cast<uint8_t>(c));
+  parallel_for(M, [&](int64_t m) {
+    const int64_t e = m_indices[m];
+    for (int64_t n = 0; n < N; ++n) {
+      if (e < 0 || e >= E) {
+        y[m * N + n] = std::nan("");
+        continue;
+      }
+      const uint8_t* wrow = qw + (e * N + n) * K;
+      const float* srow = sw + (e * NB + n / kGroup) * KB;
+      const uint8_t* arow = qa + m * K;
+      double acc = 0.0;
+      for (int64_t kb = 0; kb < KB; ++kb) {
+        double partial = 0.0;
+        for (int i = 0; i < kGroup; ++i) {
+          const int64_t k = kb * kGroup + i;
+          partial += table[arow[k]] * table[wrow[k]];
+        }
+        const double scale = static_cast<double>(sa[m * KB + kb]) * static_cast<double>(srow[kb]);
+        acc += scale * partial;
+      }
+      y[m * N + n] = acc;
+    }
+  });
+}
+
 // The magnitude sum behind the GEMM's error bound:
 //   S[m][j] = sum_k |a[m][k] * sa[m][k/128]| * |w[n][k] * sw[n/128][k/128]|
 // for n = cols[j] (all rows when null), the dequantized operands in double.

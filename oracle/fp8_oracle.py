@@ -441,3 +441,31 @@ def block_gemm_ue8m0(qA, sA8, qW, sW8, cols=None):
 
 def gemm_error_bound_ue8m0(qA, sA8, qW, sW8, cols=None, rel=1e-2):
     return gemm_error_bound(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols, rel=rel)
+
+
+# ----------------------------------------------------------------------------
+# Grouped (mixture-of-experts) GEMM ("FP8 à granularité fine", section
+# "Chemin rapide de DeepGEMM": the experts' products go through grouped
+# kernels)
+# ----------------------------------------------------------------------------
+
+def grouped_gemm(qA, sA, qW, sW, m_indices):
+    """Y[m] = the block-scaled product of token row m with the weights of its
+    expert e = m_indices[m] (qW [E, N, K], sW [E, ceil(N/128), K/128]); rows
+    with e outside [0, E) are NaN."""
+    qA = np.asarray(qA, np.uint8)
+    qW = np.asarray(qW, np.uint8)
+    sW = np.asarray(sW, np.float32)
+    mi = np.asarray(m_indices, np.int64)
+    M, K = qA.shape
+    E, N, _ = qW.shape
+    y = np.full((M, N), np.nan)
+    for e in range(E):
+        rows = np.nonzero(mi == e)[0]
+        if rows.size:
+            y[rows] = block_gemm(qA[rows], np.asarray(sA)[rows], qW[e], sW[e])
+    return y
+
+
+def grouped_gemm_ue8m0(qA, sA8, qW, sW8, m_indices):
+    return grouped_gemm(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), m_indices)

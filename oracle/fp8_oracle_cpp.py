@@ -33,6 +33,7 @@ _SIGS = {
     "orc_block_gemm": (None, [_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_sparse24_gemm": (None, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_gemm_abs_sum": (None, [_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
+    "orc_grouped_gemm": (None, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _P]),
     "orc_ue8m0_decode": (None, [_P, _I64, _P]),
     "orc_ue8m0_of_amax": (None, [_P, _I64, _P]),
     "orc_quant_act_group128_ue8m0": (None, [_P, _I64, _I64, _P, _P]),
@@ -175,6 +176,28 @@ def sparse24_gemm(qA, sA, vals, meta, sW, cols=None):
     lib().orc_sparse24_gemm(_p(qa), _p(sa), M, _p(vals), _p(meta), _p(sw), N, K, _p(c), nc,
                             _p(y))
     return y
+
+
+def grouped_gemm(qA, sA, qW, sW, m_indices):
+    """Mixture-of-experts GEMM: Y[m] = the block-scaled product of token row m
+    with the weights of its expert e = m_indices[m] (qW [E, N, K], sW
+    [E, ceil(N/128), K/128]); rows with e outside [0, E) are NaN."""
+    qa, qw = _u8(qA), _u8(qW)
+    sa = np.ascontiguousarray(np.asarray(sA, np.float32))
+    sw = np.ascontiguousarray(np.asarray(sW, np.float32))
+    mi = np.ascontiguousarray(np.asarray(m_indices, np.int32))
+    M, K = qa.shape
+    E, N, _ = qw.shape
+    if mi.shape != (M,) or sw.shape != (E, -(-N // GROUP), K // GROUP):
+        raise ValueError("grouped_gemm: shape mismatch")
+    y = np.empty((M, N), np.float64)
+    lib().orc_grouped_gemm(_p(qa), _p(sa), M, _p(qw), _p(sw), _p(mi), E, N, K, _p(y))
+    return y
+
+
+def grouped_gemm_ue8m0(qA, sA8, qW, sW8, m_indices):
+    """The grouped GEMM with UE8M0 scale codes."""
+    return grouped_gemm(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), m_indices)
 
 
 def gemm_abs_sum(qA, sA, qW, sW, cols=None):

@@ -51,7 +51,8 @@ def test_workspace_query_has_no_device_dependency(lib):
 
 
 BAD = ctypes.c_void_p(0x1000)
-MIS = ctypes.c_void_p(0x1004)
+MIS = ctypes.c_void_p(0x1004)    # 4-byte aligned only
+MIS2 = ctypes.c_void_p(0x1002)   # 2-byte aligned
 
 
 @pytest.mark.parametrize("K", [0, 100, 129, -128])
@@ -97,3 +98,22 @@ def test_fused_quantization_argument_checks(lib):
     assert g(BAD, BAD, BAD, BAD, None, BAD, BAD, 256, 128, 128, None, 0, None) == 1
     assert g(BAD, BAD, BAD, BAD, BAD, MIS, BAD, 4, 128, 128, None, 0, None) == 3
     assert g(None, None, None, None, None, None, None, 0, 128, 128, None, 0, None) == 0
+
+
+def test_grouped_and_ue8m0_argument_checks(lib):
+    """The grouped GEMMs need E >= 1 and m_indices; the UE8M0 entry points
+    follow the same shape, pointer and alignment rules; all before any launch."""
+    for g in (lib.fp8_grouped_gemm, lib.fp8_grouped_gemm_ue8m0):
+        assert g(BAD, BAD, BAD, BAD, BAD, BAD, 4, 8, 128, 0, None, 0, None) == 2     # E = 0
+        assert g(BAD, BAD, BAD, BAD, None, BAD, 4, 8, 128, 2, None, 0, None) == 1    # m_indices
+        assert g(BAD, BAD, BAD, BAD, BAD, BAD, 4, 12, 128, 2, None, 0, None) == 2    # N % 8
+        assert g(BAD, BAD, BAD, BAD, MIS2, BAD, 4, 8, 128, 2, None, 0, None) == 3    # alignment
+        assert g(BAD, MIS, BAD, MIS, MIS, BAD, 4, 8, 128, 2, None, 0, None) != 3     # 4 B is enough
+        assert g(None, None, None, None, None, None, 0, 8, 128, 2, None, 0, None) == 0
+    assert lib.fp8_block_gemm_ue8m0(BAD, BAD, BAD, BAD, BAD, 4, 8, 100, None, 0, None) == 2
+    assert lib.fp8_block_gemm_ue8m0(BAD, None, BAD, BAD, BAD, 4, 8, 128, None, 0, None) == 1
+    assert lib.fp8_quant_act_group128_ue8m0(BAD, 4, 129, BAD, BAD, None) == 2
+    assert lib.fp8_quant_weight_block128_ue8m0(MIS, 4, 128, BAD, BAD, None) == 3
+    # UE8M0 code arrays are bytes: no alignment rule (a 2-byte offset is not an error)
+    assert lib.fp8_block_gemm_ue8m0(BAD, BAD, BAD, None, BAD, 4, 8, 128, None, 0, None) == 1
+    assert lib.fp8_quant_act_group128_ue8m0(None, 0, 128, None, None, None) == 0

@@ -206,3 +206,35 @@ def test_cpp_oracle_result_does_not_depend_on_thread_count():
         np.testing.assert_array_equal(oracle.quant_weight_block128(w)[0], qw)
     finally:
         oracle.set_threads(0)
+
+
+def test_grouped_gemm_hand_computed(impl):
+    """Two experts, K = 128: a row of 1.0 codes (scale 1) against expert 0
+    (codes 1.0, scale 1) gives 128; against expert 1 (codes 1.5, scale 2)
+    128 * 1.5 * 2 = 384; a padding row (-1) has no result (NaN)."""
+    qa = np.full((3, 128), 0x38, np.uint8)
+    sa = np.ones((3, 1), np.float32)
+    qw = np.stack([np.full((8, 128), 0x38, np.uint8), np.full((8, 128), 0x3C, np.uint8)])
+    sw = np.array([[[1.0]], [[2.0]]], np.float32)
+    y = impl.grouped_gemm(qa, sa, qw, sw, np.array([0, 1, -1], np.int32))
+    np.testing.assert_array_equal(y[0], np.full(8, 128.0))
+    np.testing.assert_array_equal(y[1], np.full(8, 384.0))
+    assert np.all(np.isnan(y[2]))
+
+
+def test_grouped_gemm_reduces_to_the_dense_gemm(impl):
+    """One expert holding every row is the dense GEMM; an expert whose weights
+    are another's with every block scale times 4 gives exactly 4x its rows."""
+    x = synth.activations("deepseek", 10, 384, seed=12)
+    w = synth.weights("deepseek", 260, 384, seed=12)
+    qa, sa = impl.quant_act_group128(x)
+    qw, sw = impl.quant_weight_block128(w)
+    np.testing.assert_array_equal(
+        impl.grouped_gemm(qa, sa, qw[None], sw[None], np.zeros(10, np.int32)),
+        impl.block_gemm(qa, sa, qw, sw))
+    mi = np.array([1, 0, 0, 1, -1, 1, 0, 0, 1, 1], np.int32)
+    y = impl.grouped_gemm(qa, sa, np.stack([qw, qw]), np.stack([sw, sw * 4]), mi)
+    dense = impl.block_gemm(qa, sa, qw, sw)
+    np.testing.assert_array_equal(y[mi == 0], dense[mi == 0])
+    np.testing.assert_array_equal(y[mi == 1], 4.0 * dense[mi == 1])
+    assert np.all(np.isnan(y[mi == -1]))

@@ -396,6 +396,11 @@ def run_prefill(dev, stream, world, reps=12):
               for M in synth.PREFILL_M for kind in ("dense", "ue8m0")]
     shapes += [("sparse", 4096, N, K) for N, K in synth.SPARSE_LINEARS]
     shapes += [(kind, 8192, 4096, 14336) for kind in ("fused", "separate")]
+    # the gated MLP's gate+up GEMM with SwiGLU and the down projection's
+    # quantization fused (codes only), at decode and prefill token counts; the
+    # plain gate+up GEMM of the same shape is the dense row (or timed here)
+    shapes += [(kind, M, 28672, 4096) for M in (8, 128) for kind in ("swiglu", "dense")]
+    shapes += [("swiglu", M, 28672, 4096) for M in synth.PREFILL_M]
     rows, tot = [], {"dense": [0.0, 0.0], "ue8m0": [0.0, 0.0]}
     wcache = {}
     for kind, M, N, K in shapes:
@@ -423,6 +428,8 @@ def run_prefill(dev, stream, world, reps=12):
             y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
             qy = torch.empty(M, N, dtype=torch.uint8, device=dev)
             sy = torch.empty(M, N // 128, dtype=torch.float32, device=dev)
+            qh_sw = torch.empty(M, N // 2, dtype=torch.uint8, device=dev)
+            sh_sw = torch.empty(M, N // 256, dtype=torch.float32, device=dev)
         fns = []
         for a, s, wqq in ins:
             if kind == "dense":
@@ -436,6 +443,9 @@ def run_prefill(dev, stream, world, reps=12):
             elif kind == "fused":
                 fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_block_gemm_quant(
                     a, s, wqq[0], wqq[1], qy=qy, sy=sy, want_y=False))
+            elif kind == "swiglu":
+                fns.append(lambda a=a, s=s, wqq=wqq: fb.fp8_gemm_swiglu_quant(
+                    a, s, wqq[0], wqq[1], qh=qh_sw, sh=sh_sw, want_h=False))
             else:
                 fns.append(lambda a=a, s=s, wqq=wqq: (
                     fb.fp8_block_gemm(a, s, wqq[0], wqq[1], y=y),
@@ -446,10 +456,10 @@ def run_prefill(dev, stream, world, reps=12):
         tf = flop / (ms * 1e-3) / 1e12
         rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
                      "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4), "input_copies": n_cp})
-        if kind in tot:
+        if kind in tot and M in synth.PREFILL_M:
             tot[kind][0] += flop
             tot[kind][1] += ms
-        del fns, ins, qa, sa, wq, y, qy, sy
+        del fns, ins, qa, sa, wq, y, qy, sy, qh_sw, sh_sw
     wcache.clear()
     torch.cuda.empty_cache()
     rows += run_grouped(dev, stream, world, peak, reps)
@@ -460,7 +470,9 @@ def run_prefill(dev, stream, world, reps=12):
             "note": "dense: fp32 scales (per-K-block promotion), 2MNK FLOPs; ue8m0: power-of-two "
                     "scales applied by the block-scaled MMA; 2:4: MNK FLOPs (nonzero work) against "
                     "the dense peak; fused / separate: the down projection with the next layer's "
-                    "1x128 quantization in the epilogue / after it (not in dense_achieved); inputs "
+                    "1x128 quantization in the epilogue / after it (not in dense_achieved); "
+                    "swiglu: gate+up GEMM with SwiGLU and the down projection's quantization in "
+                    "the epilogue (codes only), against the plain gate+up GEMM; inputs "
                     "rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
 

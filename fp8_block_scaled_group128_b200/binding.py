@@ -35,6 +35,7 @@ SIGNATURES = {
     "fp8_block_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_grouped_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_grouped_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_gemm_swiglu_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
     "fp8bs_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -296,6 +297,33 @@ def fp8_grouped_gemm(qa, sa, qw, sw, m_indices, y=None, stream=None):
 def fp8_grouped_gemm_ue8m0(qa, sa8, qw, sw8, m_indices, y=None, stream=None):
     """The grouped GEMM with UE8M0 scale codes."""
     return _grouped("fp8_grouped_gemm_ue8m0", qa, sa8, qw, sw8, m_indices, y, torch.uint8, stream)
+
+
+def fp8_gemm_swiglu_quant(qa, sa, qw_gate_up, sw_gate_up, h=None, qh=None, sh=None, want_h=True,
+                          stream=None):
+    """Gate+up GEMM with SwiGLU and the down projection's 1x128 quantization
+    fused: returns (h bf16 [M, I] or None, qh uint8 [M, I], sh fp32 [M, I/128])
+    for weights [W_gate; W_up] ([2I, K])."""
+    M, K = qa.shape
+    N2 = qw_gate_up.shape[0]
+    I = N2 // 2
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa, torch.float32, (M, K // 128), "sa")
+    _dev(qw_gate_up, torch.uint8, (N2, K), "qw_gate_up")
+    _dev(sw_gate_up, torch.float32, (-(-N2 // 128), K // 128), "sw_gate_up")
+    if h is None and want_h:
+        h = _empty((M, I), torch.bfloat16, qa.device)
+    if h is not None:
+        _dev(h, torch.bfloat16, (M, I), "h")
+    qh = _empty((M, I), torch.uint8, qa.device) if qh is None else qh
+    sh = _empty((M, I // 128), torch.float32, qa.device) if sh is None else sh
+    _dev(qh, torch.uint8, (M, I), "qh")
+    _dev(sh, torch.float32, (M, I // 128), "sh")
+    _check("fp8_gemm_swiglu_quant",
+           lib().fp8_gemm_swiglu_quant(_ptr(qa), _ptr(sa), _ptr(qw_gate_up), _ptr(sw_gate_up),
+                                       _ptr(h), _ptr(qh), _ptr(sh), M, I, K, None, 0,
+                                       _stream(stream, qa)))
+    return h, qh, sh
 
 
 def get_device_error(stream=None, device=None):

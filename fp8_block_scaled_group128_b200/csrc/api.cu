@@ -326,6 +326,26 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
                                          E, wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
+int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_up,
+                          const float* sw_gate_up, void* h_bf16, void* qh_e4m3, float* sh,
+                          int64_t M, int64_t I, int64_t K, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (M < 0 || I < 0 || M > kMaxDim || I > kMaxDim / 2 || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (I % 128 != 0) return FP8BS_ERR_SHAPE;   // whole 1x128 groups of h, whole weight blocks
+  if (M == 0 || I == 0) return FP8BS_OK;
+  if (!qa || !sa || !qw_gate_up || !sw_gate_up || !qh_e4m3 || !sh) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw_gate_up) || !aligned4(sw_gate_up) ||
+      (h_bf16 && !aligned16(h_bf16)) || !aligned16(qh_e4m3) || !aligned4(sh))
+    return FP8BS_ERR_ALIGN;
+  (void)workspace;
+  (void)workspace_bytes;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_gemm_swiglu(qa, sa, qw_gate_up, sw_gate_up, h_bf16, qh_e4m3, sh, M, I, K,
+                            wait_limit(), err, static_cast<cudaStream_t>(stream));
+}
+
 int fp8bs_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FP8BS_ERR_CUDA;

@@ -105,4 +105,38 @@ int launch_block_gemm_grouped(const void* qa, const float* sa, const void* qw, c
   return launch_cfg<BN, false, false, 3, 2, 1>(ta, tb, ta, a, grid_y, 1, stream);
 }
 
+int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
+                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, long long wait_limit,
+                       int* err, cudaStream_t stream) {
+  // The prefill-order kernel for every M: a tile is 128 token rows x 128
+  // intermediate columns, i.e. gate rows [128 ct, +128) and up rows
+  // [I + 128 ct, +128) of the [2I][K] weights.
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  GemmArgs a{};
+  a.sa = sa;
+  a.sw = sw;
+  a.y = static_cast<__nv_bfloat16*>(h);
+  a.qy = static_cast<uint8_t*>(qh);
+  a.sy = sh;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(2 * I);
+  a.KB = static_cast<int>(K / 128);
+  a.NB = static_cast<int>(2 * I / 128);
+  a.swi = static_cast<int>(I);
+  a.wait_limit = wait_limit;
+  a.err = err;
+  a.row_tiles = static_cast<int>((M + 127) / 128);
+  a.col_tiles = static_cast<int>(I / 128);
+  a.splits = 1;
+  const int64_t tiles = static_cast<int64_t>(a.row_tiles) * a.col_tiles;
+  if (tiles > 0x7FFFFFFF) return FP8BS_ERR_SHAPE;
+  const int grid_y = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  const uint64_t KB = static_cast<uint64_t>(K / 128);
+  alignas(64) CUtensorMap ta, tb;
+  if (int st = encode_tmap_kblocks(&ta, qa, 128, M, KB, K, 128, 1, kSwizzle128B)) return st;
+  if (int st = encode_tmap_kblocks(&tb, qw, 128, 2 * I, KB, K, 128, 1, kSwizzle128B)) return st;
+  return launch_cfg<256, false, false, 3, 2, 1, false, true>(ta, tb, ta, a, grid_y, 1, stream);
+}
+
 }  // namespace fp8bs

@@ -46,6 +46,7 @@
 #include <map>
 #include <mutex>
 #include <tuple>
+#include <type_traits>
 
 #include "common.cuh"
 #include "e4m3_codec.cuh"
@@ -78,7 +79,17 @@ struct GemmArgs {
   // (indices outside [0, E) count as expert 0).
   const int* m_indices;
   int E;
+  // kSwiGLU: intermediate size I of a gate+up GEMM whose weights are
+  // [W_gate; W_up] ([2I][K]); y, qy, sy then hold h = silu(gate) * up
+  // ([M][I] bf16, may be null), its 1x128 codes [M][I] and scales [M][I/128].
+  int swi;
 };
+
+// silu(g) = g * sigmoid(g) = g / (1 + e^-g), in fp32 (e^-g overflowing to
+// infinity gives -0 for very negative g).
+__device__ __forceinline__ float silu_f32(float g) {
+  return g * __frcp_rn(1.0f + __expf(-g));
+}
 
 // Expert of row tile `rt` of a grouped GEMM (0 when not grouped).
 __device__ __forceinline__ int tile_expert(const GemmArgs& a, int rt) {
@@ -190,7 +201,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false,
+          bool kSwiGLU = false>
 __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>::kThreads, 1)
     block_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b,
@@ -202,6 +214,12 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
   // only if args.y is set.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
   static_assert(!kQOut || (!kSwap && C::kCols == 128), "fused quantization: one group per thread");
+  // kSwiGLU (prefill order): the 256 weight rows of a tile are gate rows
+  // [128 ct, 128 ct + 128) and up rows [I + 128 ct, ...) (two TMA boxes of 128
+  // rows); warpgroup 0 promotes the gate columns, warpgroup 1 the up columns of
+  // the same token rows, and the epilogue combines them into
+  // h = bf16(silu(gate) * up) and its 1x128 quantization along I.
+  static_assert(!kSwiGLU || (!kSwap && !kQOut && BN == 256 && kEpiWG == 2), "SwiGLU epilogue");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -324,7 +342,13 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           tma_load_3d(sm_a + stage * C::kABytes, &tmap_a, &full[stage], 0, rt * 128, kb);
           if constexpr (kSparse)
             tma_load_3d(sm_e + stage * C::kEStage, &tmap_e, &full[stage], 0, rt * 128, kb);
-          tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, brow, kb);
+          if constexpr (kSwiGLU) {
+            tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, ct * 128, kb);
+            tma_load_3d(sm_b + stage * C::kBBytes + 128 * kBK, &tmap_b, &full[stage], 0,
+                        args.swi + ct * 128, kb);
+          } else {
+            tma_load_3d(sm_b + stage * C::kBBytes, &tmap_b, &full[stage], 0, brow, kb);
+          }
         }
         __syncwarp();
         ++issued;
@@ -510,7 +534,10 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           // slot s0 + d is token row s0 + (d & 127) of the tile, weight block
           // gct * BN / 128 + (d >> 7) * kCols / 128
           const int64_t m = static_cast<int64_t>(grt) * 128 + s0 + (d & 127);
-          const int nb = (gct * BN + (d >> 7) * C::kCols) / 128;
+          // weight block of warpgroup d >> 7 (SwiGLU: the gate block, then the
+          // up block I / 128 blocks further)
+          const int nb = kSwiGLU ? ((d >> 7) == 0 ? gct : args.swi / 128 + gct)
+                                 : (gct * BN + (d >> 7) * C::kCols) / 128;
           const int kb = g_kb + sg;
           if (kb_ok && m < args.M && nb < args.NB) {
             va = args.sa[m * KB + kb];
@@ -632,7 +659,73 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
         buf ^= 1;
       }
 
-      if constexpr (!kSwap) {
+      if constexpr (kSwiGLU) {
+        // Warpgroup 0 holds gate[m][j0 + c], warpgroup 1 up[m][j0 + c] (c <
+        // 128) of token row m = 128 rt + row, in fp32. Warpgroup w turns
+        // columns [64 w, 64 w + 64) into h = bf16(silu(gate) * up): each sends
+        // the half it does not use to the other through the (here unused)
+        // output staging buffer, [2][128 rows][64] fp32 with the 16-byte
+        // chunks of a row XOR-swizzled by the row. The two halves' magnitude
+        // maxima are swapped the same way, and each warpgroup encodes its 64
+        // values with the group's scale (the activation quantizer's
+        // arithmetic on the bf16 h).
+        float* xch = reinterpret_cast<float*>(smem + C::kOffOut);
+        const int j0 = ct * 128;
+        const int64_t m = static_cast<int64_t>(rt) * 128 + row;
+        // W: this warpgroup, known at compile time so that acc stays in
+        // registers (every index below is a constant)
+        auto swiglu = [&](auto w_const) {
+          constexpr int W = decltype(w_const)::value;
+          constexpr int kSend = (1 - W) * 64;    // the half this warpgroup sends
+          float* my_row = xch + (W * 128 + row) * 64;
+          const float* peer_row = xch + ((1 - W) * 128 + row) * 64;
+          named_bar_sync(1, C::kEpiThreads);     // the previous tile's readers are done
+#pragma unroll
+          for (int c = 0; c < 64; c += 4)
+            *reinterpret_cast<float4*>(my_row + (((c >> 2) ^ (row & 15)) << 2)) =
+                make_float4(acc[kSend + c], acc[kSend + c + 1], acc[kSend + c + 2],
+                            acc[kSend + c + 3]);
+          named_bar_sync(1, C::kEpiThreads);
+          uint32_t hb[32];   // this warpgroup's 64 h values as bf16 pairs
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float4 p =
+                *reinterpret_cast<const float4*>(peer_row + (((c >> 2) ^ (row & 15)) << 2));
+            const float pv[4] = {p.x, p.y, p.z, p.w};
+            float h4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float g = W == 0 ? acc[c + i] : pv[i];
+              const float u = W == 0 ? pv[i] : acc[64 + c + i];
+              h4[i] = silu_f32(g) * u;
+            }
+            hb[c / 2] = pack_bf16x2(h4[0], h4[1]);
+            hb[c / 2 + 1] = pack_bf16x2(h4[2], h4[3]);
+          }
+          uint32_t mx = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = bf16x2_absmax(mx, hb[i]);
+          const float my_amax = absmax_to_float(mx);
+          named_bar_sync(1, C::kEpiThreads);     // every peer value has been read
+          my_row[0] = my_amax;
+          named_bar_sync(1, C::kEpiThreads);
+          const float amax = fmaxf(my_amax, peer_row[0]);
+          if (ok && m < args.M) {
+            const float sc = scale_of_amax(amax);
+            const ScaleDivider d(sc);
+            const int64_t off = m * args.swi + j0 + W * 64;
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+              const uint4 v = make_uint4(hb[c / 2], hb[c / 2 + 1], hb[c / 2 + 2], hb[c / 2 + 3]);
+              *reinterpret_cast<uint2*>(args.qy + off + c) = encode8(v, d);
+              if (args.y != nullptr) *reinterpret_cast<uint4*>(args.y + off + c) = v;
+            }
+            if (W == 0) args.sy[m * (args.swi / 128) + j0 / 128] = sc;
+          }
+        };
+        if (wg == 0) swiglu(std::integral_constant<int, 0>{});
+        else swiglu(std::integral_constant<int, 1>{});
+      } else if constexpr (!kSwap) {
         // This warpgroup's 128 columns = two 64-column boxes of the staged
         // tile. Its leader first waits until the previous tile's stores have
         // read the boxes; every thread then writes its row (16-byte chunk j
@@ -899,7 +992,8 @@ int max_active_clusters(Kern kern, int threads, int smem, int S, int dev) {
   return n;
 }
 
-template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false>
+template <int BN, bool kSwap, bool kSparse, int kStages, int kEpiWG, int kKS, bool kQOut = false,
+          bool kSwiGLU = false>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& te,
                const GemmArgs& a, int grid_y, int splits, cudaStream_t stream) {
   // (grid_y, splits) as chosen by the shape heuristic; adjusted below.
@@ -909,14 +1003,14 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
   // weight rows (plain). Without Y (a fused quantization that writes only the
   // codes) the map stays zero and is never used.
   alignas(64) CUtensorMap ty{};
-  if (a.y != nullptr) {
+  if (a.y != nullptr && !kSwiGLU) {   // the SwiGLU epilogue stores h itself
     if (int st = kSwap ? encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
                                         128, C::kChunk, kSwizzleNone)
                        : encode_tmap_2d(&ty, a.y, 2, a.N, a.M, static_cast<uint64_t>(a.N) * 2,
                                         64, 128, kSwizzle128B))
       return st;
   }
-  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS, kQOut>;
+  auto kern = block_gemm_kernel<BN, kSwap, kSparse, kStages, kEpiWG, kKS, kQOut, kSwiGLU>;
   static std::once_flag flags[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8BS_ERR_CUDA;

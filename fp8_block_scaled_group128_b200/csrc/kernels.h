@@ -35,6 +35,13 @@ int launch_block_gemm_grouped_ue8m0(const void* qa, const uint8_t* sa8, const vo
                                     int64_t N, int64_t K, int64_t E, long long wait_limit, int* err,
                                     cudaStream_t stream);
 
+// The gate+up GEMM with SwiGLU and the next layer's 1x128 quantization in its
+// epilogue: weights [W_gate; W_up] ([2I][K]); h = bf16(silu(gate) * up)
+// ([M][I], h may be null), qh [M][I], sh [M][I/128]. Returns FP8BS_* status.
+int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
+                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, long long wait_limit,
+                       int* err, cudaStream_t stream);
+
 // Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
 // N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,

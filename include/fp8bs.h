@@ -210,6 +210,28 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
                            int64_t M, int64_t N, int64_t K, int64_t E, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/*
+ * The gated MLP's gate+up GEMM with SwiGLU fused into its epilogue, keeping
+ * both block scales (TensorRT-LLM docs, performance/fp8-quantization, section
+ * "GEMM + SwiGLU Fusion in Gated-MLP": two matmuls and the SwiGLU in one
+ * kernel), and the down projection's input quantization after it:
+ *
+ *   g, u = the block-scaled GEMM of qa with the gate rows [0, I) and the up
+ *          rows [I, 2I) of qw_gate_up, in fp32;
+ *   h    = bf16_rn( silu(g) * u ),  silu(g) = g / (1 + e^-g);
+ *   qh, sh = fp8_quant_act_group128(h)   (1x128 groups along I).
+ *
+ *   qa [M][K], sa [M][K/128]           (the activations, as fp8_block_gemm)
+ *   qw_gate_up [2I][K], sw_gate_up [2I/128][K/128]  ([W_gate; W_up] quantized
+ *       with fp8_quant_weight_block128)
+ *   h_bf16 [M][I] bf16, output, may be NULL; qh_e4m3 [M][I], sh [M][I/128].
+ *   I must be a positive multiple of 128. Same errors as fp8_block_gemm.
+ */
+int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_up,
+                          const float* sw_gate_up, void* h_bf16, void* qh_e4m3, float* sh,
+                          int64_t M, int64_t I, int64_t K, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* Scratch bytes needed by the GEMMs for this shape (sparse != 0: the 2:4 GEMM). */
 size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse);
 

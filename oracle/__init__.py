@@ -29,6 +29,7 @@ from .fp8_oracle_cpp import (  # noqa: F401
     gemm_abs_sum,
     gemm_error_bound,
     gemm_error_bound_ue8m0,
+    gemm_swiglu,
     grouped_gemm,
     grouped_gemm_ue8m0,
     prune24_compress,
@@ -38,6 +39,8 @@ from .fp8_oracle_cpp import (  # noqa: F401
     quant_weight_block128_ue8m0,
     set_threads,
     sparse24_gemm,
+    swiglu,
+    swiglu_error_bound,
     threads,
     ue8m0_decode,
     ue8m0_of_amax,

@@ -451,6 +451,26 @@ void orc_grouped_gemm(const uint8_t* qa, const float* sa, int64_t M, const uint8
   });
 }
 
+// SwiGLU of the gated MLP: h = silu(g) * u with silu(g) = g / (1 + e^-g),
+// in double (g, u the gate and up outputs of the GEMM).
+void orc_swiglu(const double* g, const double* u, int64_t n, double* h) {
+  for (int64_t i = 0; i < n; ++i) h[i] = g[i] / (1.0 + std::exp(-g[i])) * u[i];
+}
+
+// Tolerance of h given tolerances tg, tu of g and u: silu has a slope of
+// magnitude below 1.1 everywhere (its derivative sigma(g) (1 + g (1 -
+// sigma(g))) lies in (-0.11, 1.1)), so
+//   |h - h_ref| <= 1.1 tg (|u| + tu) + |silu(g)| tu + 1e-5 |h|
+// with the last term for the fp32 evaluation of silu and the product.
+void orc_swiglu_bound(const double* g, const double* u, const double* tg, const double* tu,
+                      int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double sg = g[i] / (1.0 + std::exp(-g[i]));
+    out[i] = 1.1 * tg[i] * (std::fabs(u[i]) + tu[i]) + std::fabs(sg) * tu[i] +
+             1e-5 * std::fabs(sg * u[i]);
+  }
+}
+
 // The magnitude sum behind the GEMM's error bound:
 //   S[m][j] = sum_k |a[m][k] * sa[m][k/128]| * |w[n][k] * sw[n/128][k/128]|
 // for n = cols[j] (all rows when null), the dequantized operands in double.

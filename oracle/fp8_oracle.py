@@ -469,3 +469,33 @@ def grouped_gemm(qA, sA, qW, sW, m_indices):
 
 def grouped_gemm_ue8m0(qA, sA8, qW, sW8, m_indices):
     return grouped_gemm(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), m_indices)
+
+
+# ----------------------------------------------------------------------------
+# Gated MLP: SwiGLU of the gate and up outputs (TensorRT-LLM docs,
+# performance/fp8-quantization, section "GEMM + SwiGLU Fusion in Gated-MLP")
+# ----------------------------------------------------------------------------
+
+def swiglu(g, u):
+    """h = silu(g) * u with silu(g) = g / (1 + e^-g), float64."""
+    g = np.asarray(g, np.float64)
+    return g / (1.0 + np.exp(-g)) * np.asarray(u, np.float64)
+
+
+def swiglu_error_bound(g, u, tg, tu):
+    """1.1 tg (|u| + tu) + |silu(g)| tu + 1e-5 |h|: |silu'| < 1.1 everywhere."""
+    g = np.asarray(g, np.float64)
+    u = np.asarray(u, np.float64)
+    sg = g / (1.0 + np.exp(-g))
+    return 1.1 * np.asarray(tg) * (np.abs(u) + tu) + np.abs(sg) * tu + 1e-5 * np.abs(sg * u)
+
+
+def gemm_swiglu(qA, sA, qW_gate_up, sW_gate_up, rel=1e-2):
+    qW = np.asarray(qW_gate_up, np.uint8)
+    sW = np.asarray(sW_gate_up, np.float32)
+    I = qW.shape[0] // 2
+    g = block_gemm(qA, sA, qW[:I], sW[:I // GROUP])
+    u = block_gemm(qA, sA, qW[I:], sW[I // GROUP:])
+    tg = gemm_error_bound(qA, sA, qW[:I], sW[:I // GROUP], rel=rel)
+    tu = gemm_error_bound(qA, sA, qW[I:], sW[I // GROUP:], rel=rel)
+    return swiglu(g, u), swiglu_error_bound(g, u, tg, tu)

@@ -34,6 +34,8 @@ _SIGS = {
     "orc_sparse24_gemm": (None, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_gemm_abs_sum": (None, [_P, _P, _I64, _P, _P, _I64, _I64, _P, _I64, _P]),
     "orc_grouped_gemm": (None, [_P, _P, _I64, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "orc_swiglu": (None, [_P, _P, _I64, _P]),
+    "orc_swiglu_bound": (None, [_P, _P, _P, _P, _I64, _P]),
     "orc_ue8m0_decode": (None, [_P, _I64, _P]),
     "orc_ue8m0_of_amax": (None, [_P, _I64, _P]),
     "orc_quant_act_group128_ue8m0": (None, [_P, _I64, _I64, _P, _P]),
@@ -267,3 +269,41 @@ def block_gemm_ue8m0(qA, sA8, qW, sW8, cols=None):
 
 def gemm_error_bound_ue8m0(qA, sA8, qW, sW8, cols=None, rel=1e-2):
     return gemm_error_bound(qA, ue8m0_decode(sA8), qW, ue8m0_decode(sW8), cols=cols, rel=rel)
+
+
+# ------------------------------------------------------- gated MLP / SwiGLU --
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, np.float64))
+
+
+def swiglu(g, u):
+    """h = silu(g) * u, silu(g) = g / (1 + e^-g), in double."""
+    g, u = _f64(g), _f64(u)
+    h = np.empty(g.shape, np.float64)
+    lib().orc_swiglu(_p(g), _p(u), g.size, _p(h))
+    return h
+
+
+def swiglu_error_bound(g, u, tg, tu):
+    """Tolerance of h from the tolerances tg, tu of g and u (|silu'| < 1.1)."""
+    g, u, tg, tu = _f64(g), _f64(u), _f64(tg), _f64(tu)
+    out = np.empty(g.shape, np.float64)
+    lib().orc_swiglu_bound(_p(g), _p(u), _p(tg), _p(tu), g.size, _p(out))
+    return out
+
+
+def gemm_swiglu(qA, sA, qW_gate_up, sW_gate_up, rel=1e-2):
+    """The gated MLP's gate+up GEMM followed by SwiGLU: the weights are
+    [W_gate; W_up] ([2I, K], scales [2I/128, K/128]); returns (h float64
+    [M, I], its tolerance): g, u the block-scaled GEMMs with the gate and up
+    rows, h = swiglu(g, u), tolerance swiglu_error_bound with the GEMM bound
+    rel * sum |a w| of g and of u."""
+    qW = np.asarray(qW_gate_up, np.uint8)
+    sW = np.asarray(sW_gate_up, np.float32)
+    I = qW.shape[0] // 2
+    g = block_gemm(qA, sA, qW[:I], sW[:I // GROUP])
+    u = block_gemm(qA, sA, qW[I:], sW[I // GROUP:])
+    tg = gemm_error_bound(qA, sA, qW[:I], sW[:I // GROUP], rel=rel)
+    tu = gemm_error_bound(qA, sA, qW[I:], sW[I // GROUP:], rel=rel)
+    return swiglu(g, u), swiglu_error_bound(g, u, tg, tu)

@@ -117,3 +117,14 @@ def test_grouped_and_ue8m0_argument_checks(lib):
     # UE8M0 code arrays are bytes: no alignment rule (a 2-byte offset is not an error)
     assert lib.fp8_block_gemm_ue8m0(BAD, BAD, BAD, None, BAD, 4, 8, 128, None, 0, None) == 1
     assert lib.fp8_quant_act_group128_ue8m0(None, 0, 128, None, None, None) == 0
+
+
+def test_swiglu_argument_checks(lib):
+    """I must be a positive multiple of 128; codes and scales are required; h
+    is optional; M == 0 or I == 0 is a no-op."""
+    f = lib.fp8_gemm_swiglu_quant
+    assert f(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 4, 136, 128, None, 0, None) == 2
+    assert f(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 4, 128, 100, None, 0, None) == 2
+    assert f(BAD, BAD, BAD, BAD, BAD, None, BAD, 4, 128, 128, None, 0, None) == 1
+    assert f(BAD, BAD, BAD, BAD, MIS, BAD, BAD, 4, 128, 128, None, 0, None) == 3
+    assert f(None, None, None, None, None, None, None, 0, 128, 128, None, 0, None) == 0

@@ -238,3 +238,48 @@ def test_grouped_gemm_reduces_to_the_dense_gemm(impl):
     np.testing.assert_array_equal(y[mi == 0], dense[mi == 0])
     np.testing.assert_array_equal(y[mi == 1], 4.0 * dense[mi == 1])
     assert np.all(np.isnan(y[mi == -1]))
+
+
+def test_swiglu_closed_forms(impl):
+    """silu(g) = g * sigmoid(g): sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4,
+    silu(0) = 0, silu(g) -> g for large g and -> 0 for very negative g."""
+    import math
+    ln3 = math.log(3.0)
+    g = np.array([0.0, ln3, -ln3, 40.0, -800.0, 1.0])
+    u = np.array([5.0, 2.0, 2.0, 1.0, 3.0, -1.0])
+    h = impl.swiglu(g, u)
+    want = np.array([0.0, 2 * 0.75 * ln3, 2 * -0.25 * ln3, 40.0, 0.0, -1.0 / (1.0 + math.exp(-1.0))])
+    np.testing.assert_allclose(h, want, rtol=1e-15, atol=1e-300)
+    assert abs(h[4]) < 1e-300
+
+
+def test_swiglu_bound_hand_computed_and_slope_below_1_1(impl):
+    """The tolerance at g = ln 3, u = 2, tg = 0.1, tu = 0.2:
+    1.1 * 0.1 * (2 + 0.2) + (0.75 ln 3) * 0.2 + 1e-5 * (1.5 ln 3); and the
+    slope of silu, by central differences on a fine grid, stays below 1.1
+    in magnitude (the constant the bound uses)."""
+    import math
+    ln3 = math.log(3.0)
+    b = impl.swiglu_error_bound(np.array([ln3]), np.array([2.0]), np.array([0.1]), np.array([0.2]))
+    want = 1.1 * 0.1 * 2.2 + 0.75 * ln3 * 0.2 + 1e-5 * 1.5 * ln3
+    np.testing.assert_allclose(b, [want], rtol=1e-14)
+    z = np.linspace(-30, 30, 600001)
+    eps = 1e-6
+    slope = (impl.swiglu(z + eps, np.ones_like(z)) - impl.swiglu(z - eps, np.ones_like(z))) / (2 * eps)
+    assert np.abs(slope).max() < 1.1 and np.abs(slope).max() > 1.09
+
+
+def test_gemm_swiglu_hand_computed(impl):
+    """I = 128, K = 128: every activation 1.0, gate weights 1.0 with block
+    scale ln(3)/128, up weights 0.5 with scale 1/32: g = ln 3, u = 128 * 0.5
+    / 32 = 2, so h = 2 * 0.75 * ln 3 for every output."""
+    import math
+    qa = np.full((2, 128), 0x38, np.uint8)
+    sa = np.ones((2, 1), np.float32)
+    qw = np.concatenate([np.full((128, 128), 0x38, np.uint8), np.full((128, 128), 0x30, np.uint8)])
+    s_gate = np.float32(math.log(3.0) / 128)
+    sw = np.array([[s_gate], [1.0 / 32]], np.float32)
+    h, tol = impl.gemm_swiglu(qa, sa, qw, sw)
+    g = 128 * float(s_gate)
+    np.testing.assert_allclose(h, np.full((2, 128), g / (1 + math.exp(-g)) * 2.0), rtol=1e-15)
+    assert np.all(tol > 0)

@@ -8,7 +8,15 @@ seeded synthetic input generators.
 from .binding import (  # noqa: F401
     Fp8bsError,
     fp8_block_gemm,
+    fp8_block_gemm_quant,
+    fp8_block_gemm_ue8m0,
+    fp8_gather_columns,
+    fp8_gemm_swiglu_quant,
+    fp8_grouped_gemm,
+    fp8_grouped_gemm_ue8m0,
     fp8_linear,
+    fp8_quant_act_group128_ue8m0,
+    fp8_quant_weight_block128_ue8m0,
     fp8_quant_act_group128,
     fp8_quant_weight_block128,
     fp8_sparse24_gemm,

@@ -36,6 +36,7 @@ SIGNATURES = {
     "fp8_grouped_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_grouped_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_gemm_swiglu_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_gather_columns": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
     "fp8bs_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -324,6 +325,17 @@ def fp8_gemm_swiglu_quant(qa, sa, qw_gate_up, sw_gate_up, h=None, qh=None, sh=No
                                        _ptr(h), _ptr(qh), _ptr(sh), M, I, K, None, 0,
                                        _stream(stream, qa)))
     return h, qh, sh
+
+
+def fp8_gather_columns(src, dst=None, stream=None):
+    """Rank-major column shards src bf16 [P, M, Np] -> full rows dst [M, P * Np]."""
+    P, M, Np = src.shape
+    _dev(src, torch.bfloat16, (P, M, Np), "src")
+    dst = _empty((M, P * Np), torch.bfloat16, src.device) if dst is None else dst
+    _dev(dst, torch.bfloat16, (M, P * Np), "dst")
+    _check("fp8_gather_columns",
+           lib().fp8_gather_columns(_ptr(src), P, M, Np, _ptr(dst), _stream(stream, src)))
+    return dst
 
 
 def get_device_error(stream=None, device=None):

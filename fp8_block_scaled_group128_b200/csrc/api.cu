@@ -346,6 +346,19 @@ int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_u
                             wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
+int fp8_gather_columns(const void* src_bf16, int64_t P, int64_t M, int64_t Np, void* dst_bf16,
+                       void* stream) {
+  if (P < 1 || M < 0 || Np < 0 || P > kMaxDim || M > kMaxDim || Np > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (Np % 8 != 0) return FP8BS_ERR_SHAPE;   // 16-byte chunks of bf16
+  if (M == 0 || Np == 0) return FP8BS_OK;
+  if (!src_bf16 || !dst_bf16) return FP8BS_ERR_NULL;
+  if (!aligned16(src_bf16) || !aligned16(dst_bf16)) return FP8BS_ERR_ALIGN;
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  return from_cuda(launch_interleave_columns(src_bf16, P, M, Np, dst_bf16,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 int fp8bs_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FP8BS_ERR_CUDA;

@@ -42,6 +42,10 @@ int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const fl
                        void* qh, float* sh, int64_t M, int64_t I, int64_t K, long long wait_limit,
                        int* err, cudaStream_t stream);
 
+// Column shards gathered rank-major ([P][M][Np] bf16) -> full rows [M][P Np].
+cudaError_t launch_interleave_columns(const void* src, int64_t P, int64_t M, int64_t Np, void* dst,
+                                      cudaStream_t stream);
+
 // Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
 // N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,

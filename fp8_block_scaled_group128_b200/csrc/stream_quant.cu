@@ -430,3 +430,51 @@ cudaError_t launch_prune24_compress(const void* w, int64_t N, int64_t K, void* v
 }
 
 }  // namespace fp8bs
+
+namespace fp8bs {
+
+namespace {
+
+// Gathered column shards -> full rows: src [P][M][Np] (rank p's columns
+// [p Np, (p + 1) Np) of every row, as an all-gather leaves them) into
+// dst [M][P Np], 16 bytes (8 bf16) per thread, both sides coalesced.
+__global__ void __launch_bounds__(256)
+    interleave_columns_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                              int64_t P, int64_t M, int64_t np16) {
+  const int64_t total = P * M * np16;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    // i enumerates dst: row m, rank p, chunk c of that rank's columns
+    const int64_t c = i % np16;
+    const int64_t p = (i / np16) % P;
+    const int64_t m = i / (np16 * P);
+    dst[i] = src[(p * M + m) * np16 + c];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_interleave_columns(const void* src, int64_t P, int64_t M, int64_t Np, void* dst,
+                                      cudaStream_t stream) {
+  DeviceInfo dev;
+  if (current_device_info(&dev) != FP8BS_OK) return cudaErrorInvalidDevice;
+  const int64_t np16 = Np / 8;
+  const int64_t total = P * M * np16;
+  const int64_t want = (total + 255) / 256;
+  const int64_t blocks = want < 8LL * dev.sm_count ? want : 8LL * dev.sm_count;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks > 0 ? blocks : 1), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, interleave_columns_kernel, static_cast<const uint4*>(src),
+                            static_cast<uint4*>(dst), P, M, np16);
+}
+
+}  // namespace fp8bs

@@ -232,6 +232,19 @@ int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_u
                           int64_t M, int64_t I, int64_t K, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/*
+ * Output-column (N) split over P ranks (tensor parallelism; TensorRT-LLM docs,
+ * performance/fp8-quantization: the Llama-3.3-70B case study runs tensor
+ * parallel over 4 GPUs). Rank p holds weight rows [p Np, (p + 1) Np) (Np a
+ * multiple of 128, so whole 128x128 blocks) and computes those columns of Y;
+ * an all-gather over the ranks leaves them rank-major, [P][M][Np]. This call
+ * turns that into the full rows: dst[m][p Np + j] = src[p][m][j].
+ *   src_bf16 [P][M][Np], dst_bf16 [M][P Np], both bf16, no overlap;
+ *   Np a multiple of 8.
+ */
+int fp8_gather_columns(const void* src_bf16, int64_t P, int64_t M, int64_t Np, void* dst_bf16,
+                       void* stream);
+
 /* Scratch bytes needed by the GEMMs for this shape (sparse != 0: the 2:4 GEMM). */
 size_t fp8bs_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sparse);
 

@@ -128,3 +128,12 @@ def test_swiglu_argument_checks(lib):
     assert f(BAD, BAD, BAD, BAD, BAD, None, BAD, 4, 128, 128, None, 0, None) == 1
     assert f(BAD, BAD, BAD, BAD, MIS, BAD, BAD, 4, 128, 128, None, 0, None) == 3
     assert f(None, None, None, None, None, None, None, 0, 128, 128, None, 0, None) == 0
+
+
+def test_gather_columns_argument_checks(lib):
+    g = lib.fp8_gather_columns
+    assert g(BAD, 0, 4, 8, BAD, None) == 2          # P >= 1
+    assert g(BAD, 2, 4, 12, BAD, None) == 2         # Np % 8
+    assert g(None, 2, 4, 8, BAD, None) == 1
+    assert g(MIS, 2, 4, 8, BAD, None) == 3
+    assert g(None, 2, 0, 8, None, None) == 0

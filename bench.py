@@ -326,10 +326,10 @@ def barrier(world):
         dist.barrier()
 
 
-def passes_per_step(steps, pass_ms):
+def passes_per_step(steps, pass_ms, min_timed_s=MIN_TIMED_S):
     """Graph replays per counted step so that `steps` steps last at least
-    MIN_TIMED_S."""
-    return max(1, math.ceil(MIN_TIMED_S * 1e3 / (max(steps, 1) * max(pass_ms, 1e-3))))
+    `min_timed_s`."""
+    return max(1, math.ceil(min_timed_s * 1e3 / (max(steps, 1) * max(pass_ms, 1e-3))))
 
 
 def copies_beyond_l2(bytes_per_copy, cap=16):
@@ -731,7 +731,7 @@ def run_ours(args, rank, world, local):
         t1.record()
     stream.synchronize()
     pass_ms = max_over_ranks(t0.elapsed_time(t1) / 5, world)
-    passes = passes_per_step(args.steps, pass_ms)
+    passes = passes_per_step(args.steps, pass_ms, args.min_timed_s)
     total_passes = passes * args.steps
     R = min(10, total_passes)
     evented = [capture(True) for _ in range(R)]
@@ -901,6 +901,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-timed-s", type=float, default=MIN_TIMED_S,
+                    help="shortest timed region; a counted step replays the pass graph often "
+                         "enough to reach it (0: one pass per step, e.g. under a profiler)")
     ap.add_argument("--no-sections", action="store_true",
                     help="skip the prefill and quantize sections of the JSON line")
     args = ap.parse_args()

@@ -36,6 +36,7 @@ SIGNATURES = {
     "fp8_grouped_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_grouped_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_gemm_swiglu_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8bs_swiglu_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_gather_columns": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "fp8bs_get_device_error": (_I, [_P]),
@@ -301,7 +302,7 @@ def fp8_grouped_gemm_ue8m0(qa, sa8, qw, sw8, m_indices, y=None, stream=None):
 
 
 def fp8_gemm_swiglu_quant(qa, sa, qw_gate_up, sw_gate_up, h=None, qh=None, sh=None, want_h=True,
-                          stream=None):
+                          workspace=None, stream=None):
     """Gate+up GEMM with SwiGLU and the down projection's 1x128 quantization
     fused: returns (h bf16 [M, I] or None, qh uint8 [M, I], sh fp32 [M, I/128])
     for weights [W_gate; W_up] ([2I, K])."""
@@ -320,10 +321,14 @@ def fp8_gemm_swiglu_quant(qa, sa, qw_gate_up, sw_gate_up, h=None, qh=None, sh=No
     sh = _empty((M, I // 128), torch.float32, qa.device) if sh is None else sh
     _dev(qh, torch.uint8, (M, I), "qh")
     _dev(sh, torch.float32, (M, I // 128), "sh")
+    need = int(lib().fp8bs_swiglu_workspace_bytes(M, I))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=qa.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("fp8_gemm_swiglu_quant",
            lib().fp8_gemm_swiglu_quant(_ptr(qa), _ptr(sa), _ptr(qw_gate_up), _ptr(sw_gate_up),
-                                       _ptr(h), _ptr(qh), _ptr(sh), M, I, K, None, 0,
-                                       _stream(stream, qa)))
+                                       _ptr(h), _ptr(qh), _ptr(sh), M, I, K, _ptr(workspace),
+                                       ws_bytes, _stream(stream, qa)))
     return h, qh, sh
 
 

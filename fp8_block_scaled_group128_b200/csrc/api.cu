@@ -326,6 +326,11 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
                                          E, wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
+size_t fp8bs_swiglu_workspace_bytes(int64_t M, int64_t I) {
+  if (M <= 0 || I <= 0 || M > kSwiGLUDecodeMaxM) return 0;
+  return static_cast<size_t>(M) * static_cast<size_t>(2 * I) * 2;   // y [M][2I] bf16
+}
+
 int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_up,
                           const float* sw_gate_up, void* h_bf16, void* qh_e4m3, float* sh,
                           int64_t M, int64_t I, int64_t K, void* workspace,
@@ -338,12 +343,13 @@ int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_u
   if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw_gate_up) || !aligned4(sw_gate_up) ||
       (h_bf16 && !aligned16(h_bf16)) || !aligned16(qh_e4m3) || !aligned4(sh))
     return FP8BS_ERR_ALIGN;
-  (void)workspace;
-  (void)workspace_bytes;
+  const size_t need = fp8bs_swiglu_workspace_bytes(M, I);
+  if (workspace_bytes < need) return FP8BS_ERR_WORKSPACE;
+  if (need > 0 && (workspace == nullptr || !aligned16(workspace))) return FP8BS_ERR_WORKSPACE;
   int* err = device_error_word();
   if (err == nullptr) return FP8BS_ERR_CUDA;
   return launch_gemm_swiglu(qa, sa, qw_gate_up, sw_gate_up, h_bf16, qh_e4m3, sh, M, I, K,
-                            wait_limit(), err, static_cast<cudaStream_t>(stream));
+                            workspace, wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
 int fp8_gather_columns(const void* src_bf16, int64_t P, int64_t M, int64_t Np, void* dst_bf16,

@@ -203,6 +203,14 @@ __device__ __forceinline__ uint2 encode8_pow2(const uint4 v, float inv_scale) {
                     prmt(pow2_codes2(v.z, r2), pow2_codes2(v.w, r2), 0x5410u));
 }
 
+// silu(g) = g * sigmoid(g) = g / (1 + e^-g) in fp32 with the fast exponential
+// and divide (relative error below 1e-6); the exponent's argument is clamped
+// at 80 so that 1 + e^-g stays finite (for g < -80 the result is then about
+// g e^-80 instead of g e^g, both negligible next to any GEMM tolerance).
+__device__ __forceinline__ float silu_f32(float g) {
+  return __fdividef(g, 1.0f + __expf(fminf(-g, 80.0f)));
+}
+
 // bf16x2 absmax word of 8 bf16 values (see absmax_to_float).
 __device__ __forceinline__ uint32_t absmax8(const uint4 v) {
   return bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w));

@@ -106,10 +106,18 @@ int launch_block_gemm_grouped(const void* qa, const float* sa, const void* qw, c
 }
 
 int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
-                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, long long wait_limit,
-                       int* err, cudaStream_t stream) {
-  // The prefill-order kernel for every M: a tile is 128 token rows x 128
-  // intermediate columns, i.e. gate rows [128 ct, +128) and up rows
+                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, void* y_scratch,
+                       long long wait_limit, int* err, cudaStream_t stream) {
+  if (M <= kSwiGLUDecodeMaxM) {
+    // Decode-sized M: the decode-order GEMM of all 2I weight rows into the
+    // scratch y [M][2I], then SwiGLU and the quantization per 1x128 group.
+    if (int st = launch_block_gemm(qa, sa, qw, sw, y_scratch, M, 2 * I, K, wait_limit, err, stream))
+      return st;
+    return launch_swiglu_quant(y_scratch, M, I, h, qh, sh, stream) == cudaSuccess ? FP8BS_OK
+                                                                                  : FP8BS_ERR_CUDA;
+  }
+  // The prefill-order kernel with the SwiGLU epilogue: a tile is 128 token
+  // rows x 128 intermediate columns, i.e. gate rows [128 ct, +128) and up rows
   // [I + 128 ct, +128) of the [2I][K] weights.
   DeviceInfo dev;
   if (int st = current_device_info(&dev)) return st;

@@ -46,7 +46,6 @@
 #include <map>
 #include <mutex>
 #include <tuple>
-#include <type_traits>
 
 #include "common.cuh"
 #include "e4m3_codec.cuh"
@@ -85,11 +84,7 @@ struct GemmArgs {
   int swi;
 };
 
-// silu(g) = g * sigmoid(g) = g / (1 + e^-g), in fp32 (e^-g overflowing to
-// infinity gives -0 for very negative g).
-__device__ __forceinline__ float silu_f32(float g) {
-  return g * __frcp_rn(1.0f + __expf(-g));
-}
+
 
 // Expert of row tile `rt` of a grouped GEMM (0 when not grouped).
 __device__ __forceinline__ int tile_expert(const GemmArgs& a, int rt) {
@@ -591,16 +586,21 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           }
           tc_fence_after();
           const float* trow = tg + j * C::kTabStride;
-          const uint32_t taddr =
-              tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN + col0;
+          const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + tb * BN;
+          const uint32_t taddr = tlane + col0;
           if constexpr (!kSwap && C::kCols % 64 == 0) {
-            // prefill: 64 columns per TMEM round trip (two x32 loads, one wait)
-            const float sc = trow[wg * 128 + row];
+            // prefill: 64 columns per TMEM round trip (two x32 loads, one wait).
+            // SwiGLU: the tile's columns [0, 128) are gate, [128, 256) up (weight
+            // blocks 0 and 1 of the scale table); warpgroup w promotes gate and
+            // up columns [64 w, 64 w + 64) into acc[0, 64) and acc[64, 128), so a
+            // thread holds both operands of each of its outputs.
 #pragma unroll
             for (int c = 0; c < C::kCols; c += 64) {
+              const float sc = trow[(kSwiGLU ? 2 * c : wg * 128) + row];
+              const uint32_t ta = kSwiGLU ? tlane + 2 * c + wg * 64 : taddr + c;
               float v[64];
-              tmem_ld32(taddr + c, v);
-              tmem_ld32(taddr + c + 32, v + 32);
+              tmem_ld32(ta, v);
+              tmem_ld32(ta + 32, v + 32);
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 64; i += 2)
@@ -660,71 +660,49 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
       }
 
       if constexpr (kSwiGLU) {
-        // Warpgroup 0 holds gate[m][j0 + c], warpgroup 1 up[m][j0 + c] (c <
-        // 128) of token row m = 128 rt + row, in fp32. Warpgroup w turns
-        // columns [64 w, 64 w + 64) into h = bf16(silu(gate) * up): each sends
-        // the half it does not use to the other through the (here unused)
-        // output staging buffer, [2][128 rows][64] fp32 with the 16-byte
-        // chunks of a row XOR-swizzled by the row. The two halves' magnitude
-        // maxima are swapped the same way, and each warpgroup encodes its 64
-        // values with the group's scale (the activation quantizer's
+        // acc[c] = gate[m][j0 + 64 wg + c] and acc[64 + c] = up[m][j0 + 64 wg + c]
+        // (c < 64) in fp32, token row m = 128 rt + row. Each thread forms its 64
+        // h = bf16(silu(gate) * up); the scale of the 128-wide group comes from
+        // the larger of the two warpgroups' half maxima, which cross through
+        // [2][2][128] fp32 slots in the (here unused) output staging buffer. The
+        // slots alternate between tiles, so one barrier per tile separates a
+        // slot's writes from its reads and its reads from its next writes (two
+        // tiles later, after the intervening tile's barrier). Each warpgroup then
+        // encodes its 64 values with that scale (the activation quantizer's
         // arithmetic on the bf16 h).
-        float* xch = reinterpret_cast<float*>(smem + C::kOffOut);
         const int j0 = ct * 128;
         const int64_t m = static_cast<int64_t>(rt) * 128 + row;
-        // W: this warpgroup, known at compile time so that acc stays in
-        // registers (every index below is a constant)
-        auto swiglu = [&](auto w_const) {
-          constexpr int W = decltype(w_const)::value;
-          constexpr int kSend = (1 - W) * 64;    // the half this warpgroup sends
-          float* my_row = xch + (W * 128 + row) * 64;
-          const float* peer_row = xch + ((1 - W) * 128 + row) * 64;
-          named_bar_sync(1, C::kEpiThreads);     // the previous tile's readers are done
+        uint32_t hb[32];
 #pragma unroll
-          for (int c = 0; c < 64; c += 4)
-            *reinterpret_cast<float4*>(my_row + (((c >> 2) ^ (row & 15)) << 2)) =
-                make_float4(acc[kSend + c], acc[kSend + c + 1], acc[kSend + c + 2],
-                            acc[kSend + c + 3]);
-          named_bar_sync(1, C::kEpiThreads);
-          uint32_t hb[32];   // this warpgroup's 64 h values as bf16 pairs
+        for (int c = 0; c < 64; c += 2)
+          hb[c / 2] = pack_bf16x2(silu_f32(acc[c]) * acc[64 + c],
+                                  silu_f32(acc[c + 1]) * acc[64 + c + 1]);
+        uint32_t mx = 0u;
 #pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const float4 p =
-                *reinterpret_cast<const float4*>(peer_row + (((c >> 2) ^ (row & 15)) << 2));
-            const float pv[4] = {p.x, p.y, p.z, p.w};
-            float h4[4];
+        for (int i = 0; i < 32; ++i) mx = bf16x2_absmax(mx, hb[i]);
+        const float my_amax = absmax_to_float(mx);
+        float* slots = reinterpret_cast<float*>(smem + C::kOffOut) +
+                       (((tile - static_cast<int>(blockIdx.y)) / static_cast<int>(gridDim.y)) & 1) * 256;
+        slots[wg * 128 + row] = my_amax;
+        named_bar_sync(1, C::kEpiThreads);
+        const float amax = fmaxf(my_amax, slots[(1 - wg) * 128 + row]);
+        if (ok && m < args.M) {
+          const float sc = scale_of_amax(amax);
+          const ScaleDivider d(sc);
+          const int64_t off = m * args.swi + j0 + wg * 64;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float g = W == 0 ? acc[c + i] : pv[i];
-              const float u = W == 0 ? pv[i] : acc[64 + c + i];
-              h4[i] = silu_f32(g) * u;
+          for (int c = 0; c < 64; c += 16) {
+            const uint4 v0 = make_uint4(hb[c / 2], hb[c / 2 + 1], hb[c / 2 + 2], hb[c / 2 + 3]);
+            const uint4 v1 = make_uint4(hb[c / 2 + 4], hb[c / 2 + 5], hb[c / 2 + 6], hb[c / 2 + 7]);
+            const uint2 e0 = encode8(v0, d), e1 = encode8(v1, d);
+            *reinterpret_cast<uint4*>(args.qy + off + c) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+            if (args.y != nullptr) {
+              *reinterpret_cast<uint4*>(args.y + off + c) = v0;
+              *reinterpret_cast<uint4*>(args.y + off + c + 8) = v1;
             }
-            hb[c / 2] = pack_bf16x2(h4[0], h4[1]);
-            hb[c / 2 + 1] = pack_bf16x2(h4[2], h4[3]);
           }
-          uint32_t mx = 0u;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = bf16x2_absmax(mx, hb[i]);
-          const float my_amax = absmax_to_float(mx);
-          named_bar_sync(1, C::kEpiThreads);     // every peer value has been read
-          my_row[0] = my_amax;
-          named_bar_sync(1, C::kEpiThreads);
-          const float amax = fmaxf(my_amax, peer_row[0]);
-          if (ok && m < args.M) {
-            const float sc = scale_of_amax(amax);
-            const ScaleDivider d(sc);
-            const int64_t off = m * args.swi + j0 + W * 64;
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-              const uint4 v = make_uint4(hb[c / 2], hb[c / 2 + 1], hb[c / 2 + 2], hb[c / 2 + 3]);
-              *reinterpret_cast<uint2*>(args.qy + off + c) = encode8(v, d);
-              if (args.y != nullptr) *reinterpret_cast<uint4*>(args.y + off + c) = v;
-            }
-            if (W == 0) args.sy[m * (args.swi / 128) + j0 / 128] = sc;
-          }
-        };
-        if (wg == 0) swiglu(std::integral_constant<int, 0>{});
-        else swiglu(std::integral_constant<int, 1>{});
+          if (wg == 0) args.sy[m * (args.swi / 128) + j0 / 128] = sc;
+        }
       } else if constexpr (!kSwap) {
         // This warpgroup's 128 columns = two 64-column boxes of the staged
         // tile. Its leader first waits until the previous tile's stores have

@@ -38,13 +38,21 @@ int launch_block_gemm_grouped_ue8m0(const void* qa, const uint8_t* sa8, const vo
 // The gate+up GEMM with SwiGLU and the next layer's 1x128 quantization in its
 // epilogue: weights [W_gate; W_up] ([2I][K]); h = bf16(silu(gate) * up)
 // ([M][I], h may be null), qh [M][I], sh [M][I/128]. Returns FP8BS_* status.
+// Up to kSwiGLUDecodeMaxM tokens it runs as the decode GEMM into y_scratch
+// ([M][2I] bf16, 16-byte aligned) followed by the SwiGLU quantization kernel;
+// above, as one launch with the SwiGLU epilogue (y_scratch unused).
+constexpr int64_t kSwiGLUDecodeMaxM = 256;
 int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
-                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, long long wait_limit,
-                       int* err, cudaStream_t stream);
+                       void* qh, float* sh, int64_t M, int64_t I, int64_t K, void* y_scratch,
+                       long long wait_limit, int* err, cudaStream_t stream);
 
 // Column shards gathered rank-major ([P][M][Np] bf16) -> full rows [M][P Np].
 cudaError_t launch_interleave_columns(const void* src, int64_t P, int64_t M, int64_t Np, void* dst,
                                       cudaStream_t stream);
+
+// SwiGLU + 1x128 quantization of a gate+up GEMM output y [M][2I] bf16.
+cudaError_t launch_swiglu_quant(const void* y, int64_t M, int64_t I, void* h, void* qh, float* sh,
+                                cudaStream_t stream);
 
 // Dense block-scaled GEMM; with qy / sy also Y quantized in 1x128 groups along
 // N for the next layer (y may then be null when M > 256). Returns FP8BS_* status.

@@ -478,3 +478,76 @@ cudaError_t launch_interleave_columns(const void* src, int64_t P, int64_t M, int
 }
 
 }  // namespace fp8bs
+
+namespace fp8bs {
+
+namespace {
+
+// SwiGLU and the next layer's 1x128 quantization on a gate+up GEMM output:
+// y [M][2I] bf16 (gate columns [0, I), up columns [I, 2I)); per token m and
+// group j of 128 intermediate columns, h = bf16(silu(gate) * up), and codes /
+// scale of h with the activation quantizer's arithmetic. A team of 16
+// threads per group, 8 columns per thread (one 16-byte load of gate and of
+// up); no shared memory.
+__global__ void __launch_bounds__(256)
+    swiglu_quant_kernel(const __nv_bfloat16* __restrict__ y, int64_t M, int64_t I,
+                        __nv_bfloat16* __restrict__ h, uint8_t* __restrict__ qh,
+                        float* __restrict__ sh) {
+  const int64_t groups_per_row = I / 128;
+  const int64_t groups = M * groups_per_row;
+  const int64_t team = static_cast<int64_t>(blockIdx.x) * 16 + (threadIdx.x >> 4);
+  const int chunk = threadIdx.x & 15;
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const bool valid = team < groups;
+  const int64_t m = valid ? team / groups_per_row : 0;
+  const int64_t j = valid ? team - m * groups_per_row : 0;
+  uint4 g4 = make_uint4(0u, 0u, 0u, 0u), u4 = g4;
+  if (valid) {
+    const __nv_bfloat16* row = y + m * 2 * I + j * 128 + chunk * 8;
+    g4 = __ldg(reinterpret_cast<const uint4*>(row));
+    u4 = __ldg(reinterpret_cast<const uint4*>(row + I));
+  }
+  const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w}, uw[4] = {u4.x, u4.y, u4.z, u4.w};
+  uint32_t hw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float g0 = __uint_as_float(gw[i] << 16), g1 = __uint_as_float(gw[i] & 0xFFFF0000u);
+    const float u0 = __uint_as_float(uw[i] << 16), u1 = __uint_as_float(uw[i] & 0xFFFF0000u);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(silu_f32(g0) * u0, silu_f32(g1) * u1);
+    hw[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  float mx = absmax_to_float(absmax8(hv));
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  const float sc = scale_of_amax(mx);
+  if (valid) {
+    const int64_t off = m * I + j * 128 + chunk * 8;
+    reinterpret_cast<uint2*>(qh + off)[0] = encode8(hv, ScaleDivider(sc));
+    if (h != nullptr) *reinterpret_cast<uint4*>(h + off) = hv;
+    if (chunk == 0) sh[m * groups_per_row + j] = sc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_swiglu_quant(const void* y, int64_t M, int64_t I, void* h, void* qh, float* sh,
+                                cudaStream_t stream) {
+  const int64_t groups = M * (I / 128);
+  const int64_t blocks = (groups + 15) / 16;
+  if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, swiglu_quant_kernel, static_cast<const __nv_bfloat16*>(y), M, I,
+                            static_cast<__nv_bfloat16*>(h), static_cast<uint8_t*>(qh), sh);
+}
+
+}  // namespace fp8bs

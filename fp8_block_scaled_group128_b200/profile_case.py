@@ -3,7 +3,8 @@
     python -m fp8_block_scaled_group128_b200.profile_case KIND M N K ITERS
 
 KIND is one of quant_act, quant_weight, prune24, dense_gemm, sparse_gemm,
-ue8m0_gemm.
+ue8m0_gemm, swiglu (N = 2I: the gate+up GEMM with SwiGLU and the next layer's
+quantization, codes only).
 The inputs are the seeded synthetic llama tensors of that shape, prepared on
 the device by the library's own kernels before the ITERS launches of the
 kernel under test (select those with the profiler's kernel-name filter).
@@ -53,9 +54,9 @@ def main(argv):
     kind, M, N, K, iters = argv[0], int(argv[1]), int(argv[2]), int(argv[3]), int(argv[4])
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if kind in ("quant_weight", "prune24", "dense_gemm", "sparse_gemm", "ue8m0_gemm"):
+    if kind in ("quant_weight", "prune24", "dense_gemm", "sparse_gemm", "ue8m0_gemm", "swiglu"):
         w = synth.weights("llama", N, K, seed=0).to(dev)
-    if kind in ("quant_act", "dense_gemm", "sparse_gemm", "ue8m0_gemm"):
+    if kind in ("quant_act", "dense_gemm", "sparse_gemm", "ue8m0_gemm", "swiglu"):
         x = synth.activations("llama", max(M, 1), K, seed=0).to(dev)
 
     if kind == "quant_act":
@@ -80,6 +81,16 @@ def main(argv):
         else:
             vals, meta, sw, _ = fb.prune24_compress(w)
             fn = lambda: fb.fp8_sparse24_gemm(qa, sa, vals, meta, sw, y=y)  # noqa: E731
+        del w
+    elif kind == "swiglu":
+        qa, sa = fb.fp8_quant_act_group128(x)
+        qw, sw = fb.fp8_quant_weight_block128(w)
+        qh = torch.empty(M, N // 2, dtype=torch.uint8, device=dev)
+        sh = torch.empty(M, N // 256, dtype=torch.float32, device=dev)
+        need = fb.lib().fp8bs_swiglu_workspace_bytes(M, N // 2)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        fn = lambda: fb.fp8_gemm_swiglu_quant(qa, sa, qw, sw, qh=qh, sh=sh, want_h=False,  # noqa: E731
+                                              workspace=ws)
         del w
     elif kind == "ue8m0_gemm":
         qa, sa = fb.fp8_quant_act_group128_ue8m0(x)

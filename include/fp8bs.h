@@ -225,12 +225,22 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
  *   qw_gate_up [2I][K], sw_gate_up [2I/128][K/128]  ([W_gate; W_up] quantized
  *       with fp8_quant_weight_block128)
  *   h_bf16 [M][I] bf16, output, may be NULL; qh_e4m3 [M][I], sh [M][I/128].
- *   I must be a positive multiple of 128. Same errors as fp8_block_gemm.
+ *   workspace: at least fp8bs_swiglu_workspace_bytes(M, I) bytes, 16-byte
+ *       aligned (needed for M <= 256 only, else may be NULL): there the call
+ *       runs the decode-order GEMM of the 2I weight rows into this scratch
+ *       (g and u rounded to bf16) and a second kernel forms h and its codes;
+ *       for M > 256 one kernel does all of it from the fp32 accumulators.
+ *       Both forms meet the same tolerance on h.
+ *   I must be a positive multiple of 128. Same errors as fp8_block_gemm;
+ *   FP8BS_ERR_WORKSPACE for a missing or short workspace.
  */
 int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_up,
                           const float* sw_gate_up, void* h_bf16, void* qh_e4m3, float* sh,
                           int64_t M, int64_t I, int64_t K, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* Scratch bytes fp8_gemm_swiglu_quant needs for M tokens and intermediate size I. */
+size_t fp8bs_swiglu_workspace_bytes(int64_t M, int64_t I);
 
 /*
  * Output-column (N) split over P ranks (tensor parallelism; TensorRT-LLM docs,

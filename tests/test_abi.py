@@ -128,6 +128,11 @@ def test_swiglu_argument_checks(lib):
     assert f(BAD, BAD, BAD, BAD, BAD, None, BAD, 4, 128, 128, None, 0, None) == 1
     assert f(BAD, BAD, BAD, BAD, MIS, BAD, BAD, 4, 128, 128, None, 0, None) == 3
     assert f(None, None, None, None, None, None, None, 0, 128, 128, None, 0, None) == 0
+    # decode-sized M needs a scratch y [M][2I] bf16
+    assert lib.fp8bs_swiglu_workspace_bytes(8, 14336) == 8 * 2 * 14336 * 2
+    assert lib.fp8bs_swiglu_workspace_bytes(257, 14336) == 0
+    assert f(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 8, 128, 128, None, 0, None) == 4
+    assert f(BAD, BAD, BAD, BAD, BAD, BAD, BAD, 8, 128, 128, BAD, 4095, None) == 4
 
 
 def test_gather_columns_argument_checks(lib):

@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     fp8_block_gemm_ue8m0,
     fp8_gather_columns,
     fp8_gemm_swiglu_quant,
+    fp8_gemm_swiglu_quant_noalloc,
     fp8_grouped_gemm,
     fp8_grouped_gemm_ue8m0,
     fp8_linear,

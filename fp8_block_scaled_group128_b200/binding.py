@@ -18,7 +18,7 @@ FP8BS_OK = 0
 STATUS = {
     0: "FP8BS_OK", 1: "FP8BS_ERR_NULL", 2: "FP8BS_ERR_SHAPE", 3: "FP8BS_ERR_ALIGN",
     4: "FP8BS_ERR_WORKSPACE", 5: "FP8BS_ERR_CUDA", 6: "FP8BS_ERR_DEVICE_TIMEOUT",
-    7: "FP8BS_ERR_ARCH",
+    7: "FP8BS_ERR_ARCH", 8: "FP8BS_ERR_SCRATCH_LIMIT",
 }
 
 # name -> (restype, argtypes), mirroring include/fp8bs.h
@@ -36,6 +36,7 @@ SIGNATURES = {
     "fp8_grouped_gemm": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_grouped_gemm_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "fp8_gemm_swiglu_quant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "fp8_gemm_swiglu_quant_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "fp8bs_swiglu_workspace_bytes": (_SZ, [_I64, _I64]),
     "fp8_gather_columns": (_I, [_P, _I64, _I64, _I64, _P, _P]),
     "fp8bs_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
@@ -329,6 +330,29 @@ def fp8_gemm_swiglu_quant(qa, sa, qw_gate_up, sw_gate_up, h=None, qh=None, sh=No
            lib().fp8_gemm_swiglu_quant(_ptr(qa), _ptr(sa), _ptr(qw_gate_up), _ptr(sw_gate_up),
                                        _ptr(h), _ptr(qh), _ptr(sh), M, I, K, _ptr(workspace),
                                        ws_bytes, _stream(stream, qa)))
+    return h, qh, sh
+
+
+def fp8_gemm_swiglu_quant_noalloc(qa, sa, qw_gate_up, sw_gate_up, h, qh, sh, stream=None):
+    """fp8_gemm_swiglu_quant into caller-given outputs, with the library's
+    fixed device scratch in place of a workspace: this call allocates
+    nothing. h may be None; qh uint8 [M, I] and sh fp32 [M, I/128] are
+    required."""
+    M, K = qa.shape
+    N2 = qw_gate_up.shape[0]
+    I = N2 // 2
+    _dev(qa, torch.uint8, (M, K), "qa")
+    _dev(sa, torch.float32, (M, K // 128), "sa")
+    _dev(qw_gate_up, torch.uint8, (N2, K), "qw_gate_up")
+    _dev(sw_gate_up, torch.float32, (-(-N2 // 128), K // 128), "sw_gate_up")
+    if h is not None:
+        _dev(h, torch.bfloat16, (M, I), "h")
+    _dev(qh, torch.uint8, (M, I), "qh")
+    _dev(sh, torch.float32, (M, I // 128), "sh")
+    _check("fp8_gemm_swiglu_quant_noalloc",
+           lib().fp8_gemm_swiglu_quant_noalloc(_ptr(qa), _ptr(sa), _ptr(qw_gate_up),
+                                               _ptr(sw_gate_up), _ptr(h), _ptr(qh), _ptr(sh),
+                                               M, I, K, _stream(stream, qa)))
     return h, qh, sh
 
 

@@ -352,6 +352,25 @@ int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_u
                             workspace, wait_limit(), err, static_cast<cudaStream_t>(stream));
 }
 
+int fp8_gemm_swiglu_quant_noalloc(const void* qa, const float* sa, const void* qw_gate_up,
+                                  const float* sw_gate_up, void* h_bf16, void* qh_e4m3,
+                                  float* sh, int64_t M, int64_t I, int64_t K, void* stream) {
+  if (M < 0 || I < 0 || M > kMaxDim || I > kMaxDim / 2 || K > kMaxDim) return FP8BS_ERR_SHAPE;
+  if (int st = check_k(K)) return st;
+  if (I % 128 != 0) return FP8BS_ERR_SHAPE;
+  if (!swiglu_noalloc_fits(M, I)) return FP8BS_ERR_SCRATCH_LIMIT;
+  if (int st = swiglu_noalloc_setup(nullptr)) return st;   // once per device, then cached
+  if (M == 0 || I == 0) return FP8BS_OK;
+  if (!qa || !sa || !qw_gate_up || !sw_gate_up || !qh_e4m3 || !sh) return FP8BS_ERR_NULL;
+  if (!aligned16(qa) || !aligned4(sa) || !aligned16(qw_gate_up) || !aligned4(sw_gate_up) ||
+      (h_bf16 && !aligned16(h_bf16)) || !aligned16(qh_e4m3) || !aligned4(sh))
+    return FP8BS_ERR_ALIGN;
+  int* err = device_error_word();
+  if (err == nullptr) return FP8BS_ERR_CUDA;
+  return launch_gemm_swiglu_noalloc(qa, sa, qw_gate_up, sw_gate_up, h_bf16, qh_e4m3, sh, M, I, K,
+                                    wait_limit(), err, static_cast<cudaStream_t>(stream));
+}
+
 int fp8_gather_columns(const void* src_bf16, int64_t P, int64_t M, int64_t Np, void* dst_bf16,
                        void* stream) {
   if (P < 1 || M < 0 || Np < 0 || P > kMaxDim || M > kMaxDim || Np > kMaxDim) return FP8BS_ERR_SHAPE;
@@ -390,6 +409,9 @@ const char* fp8bs_status_string(int status) {
     case FP8BS_ERR_CUDA: return "CUDA call failed";
     case FP8BS_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
     case FP8BS_ERR_ARCH: return "device is not sm_100 (B200)";
+    case FP8BS_ERR_SCRATCH_LIMIT:
+      return "problem exceeds the 16 MiB device scratch of fp8_gemm_swiglu_quant_noalloc "
+             "(M <= 256 needs M * 2I * 2 bytes)";
     default: return "unknown status";
   }
 }

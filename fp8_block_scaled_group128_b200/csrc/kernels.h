@@ -46,6 +46,17 @@ int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const fl
                        void* qh, float* sh, int64_t M, int64_t I, int64_t K, void* y_scratch,
                        long long wait_limit, int* err, cudaStream_t stream);
 
+// The same with the decode path's y scratch in a fixed device array of
+// kNoAllocScratchBytes (noalloc.cu): FP8BS_ERR_SCRATCH_LIMIT when M <= 256 and
+// M * 2I * 2 bytes exceed it. swiglu_noalloc_setup looks up the array's
+// address once per device (the current one) and returns it in *scratch.
+constexpr int64_t kNoAllocScratchBytes = int64_t(16) << 20;
+int swiglu_noalloc_setup(void** scratch);
+bool swiglu_noalloc_fits(int64_t M, int64_t I);
+int launch_gemm_swiglu_noalloc(const void* qa, const float* sa, const void* qw, const float* sw,
+                               void* h, void* qh, float* sh, int64_t M, int64_t I, int64_t K,
+                               long long wait_limit, int* err, cudaStream_t stream);
+
 // Column shards gathered rank-major ([P][M][Np] bf16) -> full rows [M][P Np].
 cudaError_t launch_interleave_columns(const void* src, int64_t P, int64_t M, int64_t Np, void* dst,
                                       cudaStream_t stream);

@@ -61,7 +61,8 @@ typedef enum {
   FP8BS_ERR_WORKSPACE = 4,      /* workspace smaller than fp8bs_gemm_workspace_bytes() */
   FP8BS_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed */
   FP8BS_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up a bounded wait */
-  FP8BS_ERR_ARCH = 7            /* the current device is not sm_100 */
+  FP8BS_ERR_ARCH = 7,           /* the current device is not sm_100 */
+  FP8BS_ERR_SCRATCH_LIMIT = 8   /* the problem needs more than the fixed no-allocation scratch */
 } fp8bs_status;
 
 /*
@@ -241,6 +242,36 @@ int fp8_gemm_swiglu_quant(const void* qa, const float* sa, const void* qw_gate_u
 
 /* Scratch bytes fp8_gemm_swiglu_quant needs for M tokens and intermediate size I. */
 size_t fp8bs_swiglu_workspace_bytes(int64_t M, int64_t I);
+
+/*
+ * fp8_gemm_swiglu_quant without a workspace and without any device allocation
+ * (no cudaMalloc / cudaFree, no allocating library call). The paper (the
+ * pages this library follows) has no counterpart: it exists for callers that cannot hand over or obtain device
+ * memory per call, such as a C host that owns every buffer and passes only
+ * operands in and out (a plugin or custom-op interface with no workspace
+ * slot), or a decode loop that must not enter an allocator because
+ * cudaMalloc / cudaFree may synchronise the device and fail once a memory
+ * pool has reserved the free memory.
+ *
+ * Same operands, results and tolerance as fp8_gemm_swiglu_quant. For
+ * M <= 256 the [M][2I] bf16 intermediate lives in one fixed device array of
+ * FP8BS_NOALLOC_SCRATCH_BYTES (16 MiB) per device, reserved when the library's
+ * module is loaded; calls needing more (M <= 256 and M * 2I * 2 bytes above
+ * it: every M for I <= 16384; for I = 28672, M in 147 .. 256) return
+ * FP8BS_ERR_SCRATCH_LIMIT before anything is launched. Nothing in the array
+ * must start at zero: each call writes all of it that it reads. For M > 256
+ * no scratch is used.
+ *
+ * Setup: the first call on a device (any M, including 0, with that device
+ * current) looks up the array's address (cudaGetSymbolAddress) and caches it;
+ * make it before any stream capture. Calls on one device share the array:
+ * calls that overlap in time (other streams or host threads without ordering
+ * between them) race on it and give wrong results.
+ */
+#define FP8BS_NOALLOC_SCRATCH_BYTES (16u << 20)
+int fp8_gemm_swiglu_quant_noalloc(const void* qa, const float* sa, const void* qw_gate_up,
+                                  const float* sw_gate_up, void* h_bf16, void* qh_e4m3,
+                                  float* sh, int64_t M, int64_t I, int64_t K, void* stream);
 
 /*
  * Output-column (N) split over P ranks (tensor parallelism; TensorRT-LLM docs,

@@ -4,18 +4,15 @@
 
 KIND is one of quant_act, quant_weight, prune24, dense_gemm, sparse_gemm,
 ue8m0_gemm, swiglu (N = 2I: the gate+up GEMM with SwiGLU and the next layer's
-quantization, codes only).
-The inputs are the seeded synthetic llama tensors of that shape, prepared on
-the device by the library's own kernels before the ITERS launches of the
-kernel under test (select those with the profiler's kernel-name filter).
-Prints the mean device time of the ITERS launches (CUDA events).
-
-    python -m fp8_block_scaled_group128_b200.profile_case decode_step ITERS
-
-runs ITERS passes of the decode step's launches in issue order (the weight
-rows of the four Llama-3-8B linears, then per M in {1, 8, 32, 128} the four
-activation quantizations, dense GEMMs and 2:4 GEMMs), with about 0.9 GB on
-the device.
+quantization, codes only), grouped_gemm and grouped_ue8m0 (M routed token
+rows over 8 experts with the seeded uneven layout, each expert's rows padded
+to 128; N, K per expert).
+The inputs are the seeded synthetic llama tensors of that shape (deepseek for
+the grouped kinds), prepared on the device by the library's own kernels before
+the ITERS launches of the kernel under test (select those with the profiler's
+kernel-name filter). Prints the mean device time of the ITERS launches (CUDA
+events). One kernel and one shape per run, so that a profiler capture stays
+small.
 """
 
 import sys
@@ -26,31 +23,7 @@ from . import binding as fb
 from . import synth
 
 
-def decode_step(iters):
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    lin = synth.LLAMA3_8B_LINEARS
-    w = {nk: synth.weights("llama", *nk, seed=0).to(dev) for nk in lin}
-    x = {(M, nk): synth.activations("llama", M, nk[1], seed=0).to(dev)
-         for M in synth.DECODE_M for nk in lin}
-    for _ in range(iters):
-        q = {nk: fb.fp8_quant_weight_block128(w[nk]) for nk in lin}
-        s = {nk: fb.prune24_compress(w[nk])[:3] for nk in lin}
-        for M in synth.DECODE_M:
-            a = {nk: fb.fp8_quant_act_group128(x[(M, nk)]) for nk in lin}
-            for nk in lin:
-                fb.fp8_block_gemm(*a[nk], *q[nk])
-            for nk in lin:
-                fb.fp8_sparse24_gemm(*a[nk], *s[nk])
-    torch.cuda.synchronize()
-    if fb.get_device_error() != 0:
-        raise SystemExit("device error")
-    print(f"decode_step: {iters} passes")
-
-
 def main(argv):
-    if argv[0] == "decode_step":
-        return decode_step(int(argv[1]))
     kind, M, N, K, iters = argv[0], int(argv[1]), int(argv[2]), int(argv[3]), int(argv[4])
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -98,6 +71,30 @@ def main(argv):
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         fn = lambda: fb.fp8_block_gemm_ue8m0(qa, sa, qw, sw, y=y)  # noqa: E731
         del w
+    elif kind in ("grouped_gemm", "grouped_ue8m0"):
+        E = synth.MOE_EXPERTS
+        mi, _ = synth.moe_layout(E, M, seed=3)
+        Mp = mi.numel()
+        x = synth.activations("deepseek", Mp, K, seed=3).to(dev)
+        w = synth.expert_weights("deepseek", E, N, K, seed=3).to(dev)
+        mid = mi.to(dev)
+        qw = torch.empty(E, N, K, dtype=torch.uint8, device=dev)
+        NB, KB = -(-N // 128), K // 128
+        if kind == "grouped_gemm":
+            qa, sa = fb.fp8_quant_act_group128(x)
+            sw = torch.empty(E, NB, KB, dtype=torch.float32, device=dev)
+            for e in range(E):
+                fb.fp8_quant_weight_block128(w[e], qw=qw[e], sw=sw[e])
+            gemm = fb.fp8_grouped_gemm
+        else:
+            qa, sa = fb.fp8_quant_act_group128_ue8m0(x)
+            sw = torch.empty(E, NB, KB, dtype=torch.uint8, device=dev)
+            for e in range(E):
+                fb.fp8_quant_weight_block128_ue8m0(w[e], qw=qw[e], sw8=sw[e])
+            gemm = fb.fp8_grouped_gemm_ue8m0
+        y = torch.empty(Mp, N, dtype=torch.bfloat16, device=dev)
+        fn = lambda: gemm(qa, sa, qw, sw, mid, y=y)  # noqa: E731
+        del w, x
     else:
         raise SystemExit(f"unknown kind {kind!r}")
     torch.cuda.synchronize()
@@ -110,7 +107,8 @@ def main(argv):
     if fb.get_device_error() != 0:
         raise SystemExit("device error")
     us = e0.elapsed_time(e1) / iters * 1e3
-    extra = f", {2.0 * M * N * K / (us * 1e-6) / 1e12:.1f} TFLOP/s" if kind.endswith("gemm") else ""
+    gemm_kind = kind.endswith("gemm") or kind in ("swiglu", "grouped_ue8m0")
+    extra = f", {2.0 * M * N * K / (us * 1e-6) / 1e12:.1f} TFLOP/s" if gemm_kind else ""
     print(f"{kind} M={M} N={N} K={K}: {us:.2f} us/launch over {iters} launches{extra}")
 
 

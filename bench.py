@@ -470,9 +470,11 @@ def run_prefill(dev, stream, world, reps=12):
             "note": "dense: fp32 scales (per-K-block promotion), 2MNK FLOPs; ue8m0: power-of-two "
                     "scales applied by the block-scaled MMA; 2:4: MNK FLOPs (nonzero work) against "
                     "the dense peak; fused / separate: the down projection with the next layer's "
-                    "1x128 quantization in the epilogue / after it (not in dense_achieved); "
-                    "swiglu: gate+up GEMM with SwiGLU and the down projection's quantization in "
-                    "the epilogue (codes only), against the plain gate+up GEMM; inputs "
+                    "1x128 quantization in the epilogue / after it (M = 8192; at M <= 256 the "
+                    "fused entry point runs the GEMM and then the quantizer, two launches; not "
+                    "in dense_achieved); swiglu: gate+up GEMM with SwiGLU and the down "
+                    "projection's quantization (codes only; one kernel above 256 tokens, GEMM + "
+                    "SwiGLU kernel at or below), against the plain gate+up GEMM; inputs "
                     "rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
 

@@ -7,6 +7,22 @@ namespace fp8bs {
 
 using namespace gemm_detail;
 
+// Operand order of a dense GEMM. Up to 256 tokens the weights go on the MMA M
+// side (decode order: the HBM-bound weight stream spread over the SMs, split
+// over K where the tiles alone do not fill them). From 65 tokens on, a weight
+// matrix wide enough to give the prefill-order kernel (128 tokens x 256 weight
+// rows per tile) at least three quarters of a wave of tiles runs in prefill
+// order instead: its promotion applies one scale per row, where the decode
+// order's 128 x 128 tiles apply one per column, which paces them at 128 tokens
+// (gate+up of Llama-3-8B at M = 128: HBM-bound per SM at ~36 GB/s in decode
+// order).
+inline bool decode_order(int64_t M, int64_t N, int sm_count) {
+  if (M > 256) return false;
+  if (M <= 64) return true;
+  const int64_t prefill_tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  return 4 * prefill_tiles < 3 * static_cast<int64_t>(sm_count);
+}
+
 int launch_block_gemm(const void* qa, const float* sa, const void* qw, const float* sw, void* y,
                       int64_t M, int64_t N, int64_t K, long long wait_limit, int* err,
                       cudaStream_t stream, void* qy, float* sy) {
@@ -27,7 +43,7 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   alignas(64) CUtensorMap ta, tb;
 
   const uint64_t KB = static_cast<uint64_t>(K / 128);
-  if (M <= 256 && qy != nullptr) {
+  if (decode_order(M, N, dev.sm_count) && qy != nullptr) {
     // Decode-sized M with the next layer's quantization: Y, then the
     // activation quantizer on it (the decode-order tile holds a group of N
     // across four warps, or across a cluster with a K split).
@@ -37,7 +53,7 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
     return launch_quant_act_group128(y, M, N, qy, sy, stream) == cudaSuccess ? FP8BS_OK
                                                                               : FP8BS_ERR_CUDA;
   }
-  if (M <= 256) {
+  if (decode_order(M, N, dev.sm_count)) {
     // Decode: weights on the MMA M side, tokens on the MMA N side; stages of
     // two K-blocks.
     constexpr int kKS = 2;
@@ -108,7 +124,9 @@ int launch_block_gemm_grouped(const void* qa, const float* sa, const void* qw, c
 int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
                        void* qh, float* sh, int64_t M, int64_t I, int64_t K, void* y_scratch,
                        long long wait_limit, int* err, cudaStream_t stream) {
-  if (M <= kSwiGLUDecodeMaxM) {
+  DeviceInfo dev;
+  if (int st = current_device_info(&dev)) return st;
+  if (M <= kSwiGLUDecodeMaxM && decode_order(M, 2 * I, dev.sm_count)) {
     // Decode-sized M: the decode-order GEMM of all 2I weight rows into the
     // scratch y [M][2I], then SwiGLU and the quantization per 1x128 group.
     if (int st = launch_block_gemm(qa, sa, qw, sw, y_scratch, M, 2 * I, K, wait_limit, err, stream))
@@ -118,9 +136,7 @@ int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const fl
   }
   // The prefill-order kernel with the SwiGLU epilogue: a tile is 128 token
   // rows x 128 intermediate columns, i.e. gate rows [128 ct, +128) and up rows
-  // [I + 128 ct, +128) of the [2I][K] weights.
-  DeviceInfo dev;
-  if (int st = current_device_info(&dev)) return st;
+  // [I + 128 ct, +128) of the [2I][K] weights (y_scratch unused).
   GemmArgs a{};
   a.sa = sa;
   a.sw = sw;

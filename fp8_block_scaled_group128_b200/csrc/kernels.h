@@ -38,9 +38,10 @@ int launch_block_gemm_grouped_ue8m0(const void* qa, const uint8_t* sa8, const vo
 // The gate+up GEMM with SwiGLU and the next layer's 1x128 quantization in its
 // epilogue: weights [W_gate; W_up] ([2I][K]); h = bf16(silu(gate) * up)
 // ([M][I], h may be null), qh [M][I], sh [M][I/128]. Returns FP8BS_* status.
-// Up to kSwiGLUDecodeMaxM tokens it runs as the decode GEMM into y_scratch
-// ([M][2I] bf16, 16-byte aligned) followed by the SwiGLU quantization kernel;
-// above, as one launch with the SwiGLU epilogue (y_scratch unused).
+// Up to kSwiGLUDecodeMaxM tokens it may run as the decode GEMM into y_scratch
+// ([M][2I] bf16, 16-byte aligned) followed by the SwiGLU quantization kernel
+// (when the dense GEMM's dispatch picks the decode order for N = 2I);
+// otherwise as one launch with the SwiGLU epilogue (y_scratch unused).
 constexpr int64_t kSwiGLUDecodeMaxM = 256;
 int launch_gemm_swiglu(const void* qa, const float* sa, const void* qw, const float* sw, void* h,
                        void* qh, float* sh, int64_t M, int64_t I, int64_t K, void* y_scratch,

@@ -133,9 +133,10 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
  * y, and qy / sy = fp8_quant_act_group128(y) of that bf16 y, i.e. y's rows
  * cut into 1x128 groups along N ("FP8 à granularité fine": the output of one
  * linear is the activation of the next, quantized per token per 128
- * channels). For M > 256 the GEMM's epilogue quantizes its own tile (each
- * promotion thread holds one group); for M <= 256 y is written and then
- * quantized by the activation quantizer.
+ * channels). When the GEMM runs in prefill order (M > 256, or M > 64 with N
+ * wide enough to fill most of the GPU with 128 x 256 tiles) its epilogue
+ * quantizes its own tile (each promotion thread holds one group); otherwise
+ * y is written and then quantized by the activation quantizer.
  *
  *   y_bf16  [M][N] bf16, output; may be NULL when M > 256 (then only the codes
  *           are written), required when M <= 256.
@@ -227,11 +228,12 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
  *       with fp8_quant_weight_block128)
  *   h_bf16 [M][I] bf16, output, may be NULL; qh_e4m3 [M][I], sh [M][I/128].
  *   workspace: at least fp8bs_swiglu_workspace_bytes(M, I) bytes, 16-byte
- *       aligned (needed for M <= 256 only, else may be NULL): there the call
- *       runs the decode-order GEMM of the 2I weight rows into this scratch
- *       (g and u rounded to bf16) and a second kernel forms h and its codes;
- *       for M > 256 one kernel does all of it from the fp32 accumulators.
- *       Both forms meet the same tolerance on h.
+ *       aligned (required for M <= 256 only, else may be NULL): there the
+ *       call may run the decode-order GEMM of the 2I weight rows into this
+ *       scratch (g and u rounded to bf16) and a second kernel that forms h and
+ *       its codes; otherwise (M > 256, or a 2I wide enough for the prefill
+ *       order as in fp8_block_gemm_quant) one kernel does all of it from the
+ *       fp32 accumulators. Both forms meet the same tolerance on h.
  *   I must be a positive multiple of 128. Same errors as fp8_block_gemm;
  *   FP8BS_ERR_WORKSPACE for a missing or short workspace.
  */

@@ -161,6 +161,41 @@ def test_ragged_shapes(M, N, K):
     assert stats["max_err_over_sum"] < 1e-4
 
 
+@pytest.mark.parametrize("M", [64, 65, 128, 200, 256])
+def test_operand_order_boundary_wide_n(M):
+    """At 65..256 tokens a weight matrix wide enough for three quarters of a
+    wave of 128 x 256 prefill tiles runs in prefill order, below 65 tokens in
+    decode order: both sides of the switch, a half-filled second row tile
+    (200) and a full one (256), on a 28672-row (gate+up) weight with a ragged
+    last column tile avoided by N % 256 == 0 and a short K."""
+    N, K = 28672, 512
+    stats = _chain_case("llama", M, N, K, seed=30 + M, rows=_sample(M, 24, M, must=(0, M - 1)),
+                        blocks=_blocks(N, 12, M))
+    assert stats["max_err_over_sum"] < 1e-4
+
+
+@pytest.mark.parametrize("M,N", [(65, 28672), (200, 14208), (128, 28288), (128, 28160)])
+def test_fused_quantization_in_prefill_order_at_decode_sizes(M, N):
+    """fp8_block_gemm_quant for 65..256 tokens on wide weights. On 148 SMs:
+    N = 28288 at M = 128 is the narrowest width that takes the one-kernel
+    prefill-order form (111 tiles of 128 x 256) and 28160 the widest that
+    stays in decode order (GEMM, then the quantizer); 28288 and 14208 (M = 200,
+    two row tiles) leave the last 256-column tile half empty. y equal to
+    fp8_block_gemm's, codes and scales equal to the oracle's quantization of
+    that y."""
+    K = 384
+    qa, sa, qw, sw = _quantized("llama", M, N, K, 5)
+    args = [to_dev(a) for a in (qa, sa, qw, sw)]
+    y_plain = fb.fp8_block_gemm(*args)
+    y, qy, sy = fb.fp8_block_gemm_quant(*args)
+    torch.cuda.synchronize()
+    assert fb.get_device_error() == 0
+    assert torch.equal(y, y_plain)
+    q_ref, s_ref = oracle.quant_act_group128(y.cpu())
+    np.testing.assert_array_equal(qy.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(sy.cpu().numpy(), s_ref)
+
+
 def test_zero_scales_and_extreme_values():
     M, N, K = 40, 272, 512
     x = synth.activations("deepseek", M, K, seed=7).float().numpy()

@@ -77,6 +77,17 @@ def test_llama3_8b_decode(M):
     assert _swiglu_case(M, I, 4096, seed=20 + M, groups=_sample(I // 128, 10, M, must=(0, 111))) <= 1.0
 
 
+@pytest.mark.parametrize("M", [64, 65, 200])
+def test_two_forms_at_the_switch(M):
+    """At most 256 tokens the call takes the decode form (GEMM into the
+    workspace, then the SwiGLU kernel) only where the dense dispatch keeps the
+    decode order for N = 2I; with I = 14336 that is M <= 64, and M = 65 and 200
+    (two row tiles, the second partial) run the one-kernel form. K = 512."""
+    I = 14336
+    assert _swiglu_case(M, I, 512, seed=40 + M, rows=_sample(M, 24, M, must=(0, M - 1)),
+                        groups=_sample(I // 128, 10, M, must=(0, 111))) <= 1.0
+
+
 @pytest.mark.parametrize("M", [2048, 8192])
 def test_llama3_8b_prefill(M):
     I = 14336

@@ -67,16 +67,16 @@ struct ScaleDivider {
   float r;
   bool fast;       // Markstein allowed (per element checks still apply)
   bool fast_all;   // branch-free codes allowed for every element (see codes2)
-  uint64_t r2;     // (r, r) packed for fp32x2 arithmetic
-  uint64_t ns2;    // (-s, -s)
+  uint64_t nr2;    // (-r, -r) packed for fp32x2 arithmetic
+  uint64_t s2;     // (s, s)
 
   __device__ __forceinline__ explicit ScaleDivider(float scale) : s(scale) {
     r = __frcp_rn(scale);
     // s normal (>= 2^-126) keeps r finite and normal for every bf16 amax.
     fast = scale >= 1.17549435e-38f && scale <= 1.0e37f;
     fast_all = scale >= 8.27180613e-25f && scale <= 1.0e37f;  // s >= 2^-80
-    r2 = pack_f32x2(r, r);
-    ns2 = pack_f32x2(-scale, -scale);
+    nr2 = pack_f32x2(-r, -r);
+    s2 = pack_f32x2(scale, scale);
   }
 
   // Markstein's quotient without the range checks.
@@ -86,10 +86,15 @@ struct ScaleDivider {
     return __fmaf_rn(e, r, q0);
   }
 
-  // The same on two values at once (fp32x2 instructions; each lane rounds
-  // exactly like the scalar form, since q0 * (-s) + x == -q0 * s + x).
-  __device__ __forceinline__ void quotient2_unchecked(float x0, float x1, float& q0,
-                                                      float& q1) const {
+  // -(x / s) of two values at once, Markstein's steps on -r = -1/s (fp32x2
+  // instructions): q' = RN(x * -r), e = RN(q' * s + x), RN(e * -r + q'). For
+  // x != 0 every step is the exact negation of the scalar form's (round to
+  // nearest is symmetric: q' = -q0, e is the same residual, the result -q).
+  // For x = +-0 the result is the zero of the opposite sign as well: the
+  // residual is +0 (opposite zeros add to +0) and the last sum, -0 + -0 for
+  // x = +0 and -0 + +0 for x = -0, rounds to -0 and +0.
+  __device__ __forceinline__ void neg_quotient2_unchecked(float x0, float x1, float& q0,
+                                                         float& q1) const {
     asm("{\n\t.reg .b64 x, q, e;\n\t"
         "mov.b64 x, {%2, %3};\n\t"
         "mul.rn.f32x2 q, x, %4;\n\t"
@@ -97,30 +102,27 @@ struct ScaleDivider {
         "fma.rn.f32x2 q, e, %4, q;\n\t"
         "mov.b64 {%0, %1}, q;\n\t}"
         : "=f"(q0), "=f"(q1)
-        : "f"(x0), "f"(x1), "l"(r2), "l"(ns2));
+        : "f"(x0), "f"(x1), "l"(nr2), "l"(s2));
   }
 
-  // E4M3 codes of the magnitudes of two bf16 values packed as (lo, hi) halves
-  // of w (lo -> byte 0), through the unchecked quotient (fast_all only).
-  __device__ __forceinline__ uint32_t mag_codes2(uint32_t w) const {
-    const uint32_t a = w & 0x7FFF7FFFu;
+  // E4M3 codes of two bf16 values packed as (lo, hi) halves of w (lo -> byte
+  // 0) with their sign bits inverted: the conversion of -(x / s) (E4M3
+  // rounding and saturation are symmetric, so only the sign bit differs from
+  // the code of x / s, zeros included). fast_all only.
+  __device__ __forceinline__ uint32_t flipped_codes2(uint32_t w) const {
     float q0, q1;
-    quotient2_unchecked(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u), q0, q1);
+    neg_quotient2_unchecked(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u), q0, q1);
     return __nv_cvt_float2_to_fp8x2(make_float2(q0, q1), __NV_SATFINITE, __NV_E4M3);
   }
 
   // E4M3 codes of two bf16 values packed as (lo, hi) halves of w, for s > 0
-  // (x0 = lo -> byte 0). With s >= 2^-80 both elements go through the
-  // unchecked quotient of their magnitudes and take their sign bit from the
-  // input: the quotient is exact where it can be nonzero in E4M3 (|x| >=
+  // (x0 = lo -> byte 0). With s >= 2^-80 both elements take the branch-free
+  // path: the quotient is exact where it can be nonzero in E4M3 (|x| >=
   // 2^-100 and |x / s| >= 2^-100), and everywhere else it is below 2^-20, far
-  // under the smallest E4M3 subnormal, so the code is the signed zero either
-  // way. Smaller scales take the checked path.
+  // under the smallest E4M3 subnormal, so the code is the zero of x's sign
+  // either way. Smaller scales take the checked path.
   __device__ __forceinline__ uint32_t codes2(uint32_t w) const {
-    if (fast_all) {
-      // byte 0 <- sign of the low bf16 (bit 15), byte 1 <- sign of the high one
-      return mag_codes2(w) | (prmt(w, 0u, 0x44B9u) & 0x8080u);
-    }
+    if (fast_all) return flipped_codes2(w) ^ 0x8080u;
     const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
     return __nv_cvt_float2_to_fp8x2(make_float2((*this)(x0), (*this)(x1)), __NV_SATFINITE,
                                     __NV_E4M3);
@@ -128,10 +130,7 @@ struct ScaleDivider {
 
   // Four codes: the two of w0 in bytes 0-1, the two of w1 in bytes 2-3.
   __device__ __forceinline__ uint32_t codes4(uint32_t w0, uint32_t w1) const {
-    if (fast_all) {
-      // the four input sign bits (bits 15, 31 of w0 and of w1), replicated
-      return prmt(mag_codes2(w0), mag_codes2(w1), 0x5410u) | (prmt(w0, w1, 0xFDB9u) & 0x80808080u);
-    }
+    if (fast_all) return prmt(flipped_codes2(w0), flipped_codes2(w1), 0x5410u) ^ 0x80808080u;
     return prmt(codes2(w0), codes2(w1), 0x5410u);
   }
 

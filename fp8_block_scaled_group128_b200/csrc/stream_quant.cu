@@ -50,6 +50,20 @@ struct QArgs {
   int* err;
 };
 
+// |x| of both bf16 halves, and the lane mask of a >= b (0xFFFF per 16-bit
+// lane where it holds), both on the half-precision pipe.
+__device__ __forceinline__ uint32_t abs_bf16x2(uint32_t x) {
+  uint32_t d;
+  asm("abs.bf16x2 %0, %1;" : "=r"(d) : "r"(x));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t ge_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // 2:4 selection, metadata and codes of the 8 weights (two groups of 4 along
 // K) in one 16-byte chunk: group 0 in v.x (elements 0, 1) and v.y (2, 3),
 // group 1 in v.z and v.w. Element j "beats" element i when |w_j| > |w_i|, or
@@ -57,10 +71,12 @@ struct QArgs {
 // it, which keeps exactly two per group.
 //
 // Both groups are ranked at once in 16-bit lanes: E_j pairs element j of
-// group 0 (low half) with element j of group 1 (high half); for i < j,
-// (E_i | 0x8000 per lane) - |E_j| leaves bit 15 of each lane set exactly when
-// |w_i| >= |w_j| (15-bit magnitudes, no borrow between the lanes). Each kept
-// flag is then the majority of three such bits.
+// group 0 (low half) with element j of group 1 (high half); for i < j a
+// packed bf16 comparison of the magnitudes (abs.bf16x2, set.ge.u32.bf16x2 on
+// the half-precision pipe, which leaves the integer pipe to the rest) gives
+// 0xFFFF in each lane where |w_i| >= |w_j|: for finite values the order of the
+// magnitudes as numbers is that of their 15-bit patterns, and +0 and -0 tie.
+// Each kept flag is then the majority of three such masks.
 //
 // Returns the 4 value bytes (kept codes of group 0 in position order, then
 // group 1); sets the metadata byte (group 0 nibble in bits 0-3, group 1 in
@@ -70,28 +86,27 @@ __device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d,
                                            uint4& pruned) {
   const uint32_t e0 = prmt(v.x, v.z, 0x5410u), e1 = prmt(v.x, v.z, 0x7632u);
   const uint32_t e2 = prmt(v.y, v.w, 0x5410u), e3 = prmt(v.y, v.w, 0x7632u);
-  constexpr uint32_t kTop = 0x80008000u;
-  const uint32_t g0 = e0 | kTop, g1 = e1 | kTop, g2 = e2 | kTop, g3 = e3 | kTop;
-  // c_ij (bit 15 / 31): |w_i| >= |w_j|, i.e. i beats j (i < j); per lane
-  // (0x8000 + |w_i|) - (0x8000 + |w_j|) + 0x8000
-  const uint32_t c01 = g0 - g1 + kTop, c02 = g0 - g2 + kTop, c03 = g0 - g3 + kTop;
-  const uint32_t c12 = g1 - g2 + kTop, c13 = g1 - g3 + kTop, c23 = g2 - g3 + kTop;
+  const uint32_t g0 = abs_bf16x2(e0), g1 = abs_bf16x2(e1), g2 = abs_bf16x2(e2),
+                 g3 = abs_bf16x2(e3);
+  // c_ij (each lane all ones or zero): |w_i| >= |w_j|, i.e. i beats j (i < j)
+  const uint32_t c01 = ge_bf16x2(g0, g1), c02 = ge_bf16x2(g0, g2), c03 = ge_bf16x2(g0, g3);
+  const uint32_t c12 = ge_bf16x2(g1, g2), c13 = ge_bf16x2(g1, g3), c23 = ge_bf16x2(g2, g3);
   auto maj = [](uint32_t a, uint32_t b, uint32_t c) { return (a & b) | (a & c) | (b & c); };
   const uint32_t k0 = maj(c01, c02, c03);      // kept: beaten at most once
   const uint32_t k1 = maj(~c01, c12, c13);
   const uint32_t k2 = maj(~c02, ~c12, c23);
   const uint32_t k3 = maj(~c03, ~c13, ~c23);
-  // nibble bits: i0 = 0 | 1 | 2 (first kept), i1 = 1 | 2 | 3 (last kept)
-  const uint32_t b0 = ~k0 & k1 & kTop;          // i0 bit 0
-  const uint32_t b1 = ~k0 & ~k1 & kTop;         // i0 bit 1
-  const uint32_t b2 = (k3 | ~k2) & kTop;        // i1 bit 0
-  const uint32_t b3 = (k3 | k2) & kTop;         // i1 bit 1
-  // i0 and i1 of group 0 in bits 0-1 and 8-9, of group 1 in bits 16-17 and
-  // 24-25
-  const uint32_t sp = (b0 >> 15) | (b1 >> 14) | (b2 >> 7) | (b3 >> 6);
-  // nibbles i0 | i1 << 2: group 0 in bits 0-3, group 1 in bits 16-19
-  const uint32_t nib = sp | (sp >> 6);
-  meta = (nib & 0xFu) | ((nib >> 12) & 0xF0u);
+  // i0 = 0 | 1 | 2 (first kept), i1 = 1 | 2 | 3 (last kept); the flags are
+  // whole-lane masks, so each index bit is placed by its own constant: i0 and
+  // i1 of group 0 in bits 0-1 and 8-9, of group 1 in bits 16-17 and 24-25
+  const uint32_t sp = ((~k0 & k1 & 0x00010001u) | (~k0 & ~k1 & 0x00020002u)) |
+                      (((k3 | ~k2) & 0x01000100u) | ((k3 | k2) & 0x02000200u));
+  // metadata byte: nibbles i0 | i1 << 2 of group 0 in bits 0-3, of group 1 in
+  // bits 4-7. sp * (1 + 2^6 + 2^12 + 2^18) adds four shifted copies of sp: the
+  // fields at bits 0, 8, 16 and 24 land at bits 18, 20, 22 and 24, no two
+  // partial sums overlap below bit 26 (so nothing carries into them), and the
+  // byte is bits 18-25 (the caller stores the low 8 bits).
+  meta = (sp * 0x41041u) >> 18;
   // kept bf16 values of each group in position order (halfwords i0 and i1):
   // byte selector 2i0 | (2i0 + 1) << 4 | 2i1 << 8 | (2i1 + 1) << 12, of which
   // prmt reads only the low 16 bits

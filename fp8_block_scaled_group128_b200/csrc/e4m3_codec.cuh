@@ -79,13 +79,6 @@ struct ScaleDivider {
     s2 = pack_f32x2(scale, scale);
   }
 
-  // Markstein's quotient without the range checks.
-  __device__ __forceinline__ float quotient_unchecked(float x) const {
-    const float q0 = __fmul_rn(x, r);
-    const float e = __fmaf_rn(-q0, s, x);
-    return __fmaf_rn(e, r, q0);
-  }
-
   // -(x / s) of two values at once, Markstein's steps on -r = -1/s (fp32x2
   // instructions): q' = RN(x * -r), e = RN(q' * s + x), RN(e * -r + q'). For
   // x != 0 every step is the exact negation of the scalar form's (round to

@@ -91,7 +91,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
-// mbar_wait by every lane of a warp with one verdict for all: the warp stays
+// mbar_wait by every lane of a warp with one result for all: the warp stays
 // converged even when the limit runs out for some lanes only.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, long long limit) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit));

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_tiles = args.row_tiles * args.col_tiles;
   const int KB = args.KB;
   const long long limit = args.wait_limit;
-  // the abort flag as one verdict for the whole warp (keeps role loops converged)
+  // the abort flag as one result for the whole warp (keeps role loops converged)
   auto aborted = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0); };
 
   if (threadIdx.x == 0) {

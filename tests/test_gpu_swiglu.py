@@ -5,7 +5,7 @@ The GPU quantizes x and [W_gate; W_up] and runs the fused GEMM. The oracle
 quantizes, from the same bf16 inputs, the compared token rows and the gate /
 up weight blocks of the compared intermediate columns (asserting the GPU's
 bytes equal its own), computes h = silu(g) * u in double and its tolerance
-(the task's GEMM bound on g and on u, carried through silu's slope < 1.1),
+(the GEMM parity bound 1e-2 sum|a w| on g and on u, carried through silu's slope < 1.1),
 and h must be within that plus one bf16 ulp. The codes and scales of h must
 equal the oracle's 1x128 quantization of the GPU's own bf16 h, bit for bit."""
 

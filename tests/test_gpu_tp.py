@@ -36,7 +36,7 @@ def test_gather_columns_is_the_rank_major_transpose(P, M, Np):
 @pytest.mark.parametrize("M,N,K,P", [(512, 4096, 4096, 4), (8, 6144, 4096, 4), (130, 1024, 512, 2)])
 def test_shards_on_one_gpu_reassemble_the_full_gemm(M, N, K, P):
     """Each shard's GEMM written into its slot of the rank-major buffer, then
-    interleaved, equals the oracle's full product within the task's bound
+    interleaved, equals the oracle's full product within the GEMM parity bound
     (prefill order: also byte-equal to the unsplit GEMM)."""
     x = synth.activations("llama", M, K, seed=5)
     w = synth.weights("llama", N, K, seed=5)

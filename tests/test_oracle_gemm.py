@@ -130,7 +130,7 @@ def test_error_bound_hand_computed(impl):
     qa, sa, qw, sw = _two_by_two_operands()
     np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, rel=1.0),
                                   [[192.0, 64.0], [6.0, 0.0]])
-    # the default rel is the task's 1e-2
+    # the default rel is the parity bound's 1e-2
     np.testing.assert_allclose(impl.gemm_error_bound(qa, sa, qw, sw),
                                [[1.92, 0.64], [0.06, 0.0]], rtol=1e-15)
     np.testing.assert_array_equal(impl.gemm_error_bound(qa, sa, qw, sw, cols=[1], rel=1.0),

@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
         if (i * (kQThreads / 16) >= rows_here) break;
         const int64_t r = r0 + i * (kQThreads / 16);
         if constexpr (kMode == QMode::kWeight) {
-          reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8(v[i], d);
+          reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8_sign_merged(v[i], d);
         } else {
           constexpr bool kOut = kMode == QMode::kPruneOut;
           uint32_t meta;

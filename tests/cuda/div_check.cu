@@ -3,7 +3,8 @@
 // s = fl32(amax / 448) for every positive finite bf16 amax, and every finite
 // bf16 x with |x| <= amax (both signs). Also checks the E4M3 codes, both of
 // the checked quotient and of the quantizers' branch-free pair path (both
-// halves of the pair), and the quantizers' scale amax / 448 for every amax.
+// halves of the pair, the four-code forms), and the quantizers' scale
+// amax / 448 for every amax.
 #include <cstdint>
 
 #include "../../fp8_block_scaled_group128_b200/csrc/e4m3_codec.cuh"
@@ -50,6 +51,8 @@ __global__ void div_check_kernel(Result* res) {
     // four at once: (x, -x) in the first word, (-x, x) in the second
     const uint32_t c4 = d.codes4((xb << 16) | (xb ^ 0x8000u), ((xb ^ 0x8000u) << 16) | xb);
     bad_c += (c4 != (c2p | ((((c2p & 0xFFu) << 8) | (c2p >> 8)) << 16)));
+    // the weight-block kernel's form of the same four codes
+    bad_c += (d.codes4_sign_merged((xb << 16) | (xb ^ 0x8000u), ((xb ^ 0x8000u) << 16) | xb) != c4);
     const uint32_t cn_ref =
         __nv_cvt_float_to_fp8(__fdiv_rn(-x, s), __NV_SATFINITE, __NV_E4M3);
     bad_c += (c != c_ref) + (c2 != c_ref) + ((c2p >> 8) != c_ref) + ((c2p & 0xFFu) != cn_ref);

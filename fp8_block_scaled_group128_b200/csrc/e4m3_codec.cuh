@@ -54,7 +54,9 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
 // s = fl32(amax / 448), correctly rounded, for a finite amax >= 0.
 __device__ __forceinline__ float scale_of_amax(float amax) {
   if (amax >= 7.88860905e-31f) {  // 2^-100: quotient and residual stay normal
-    const float r = __frcp_rn(448.0f);
+    // 1/448 = 2^-9 * 8/7 rounded to nearest: mantissa 8/7 * 2^23 =
+    // 9586980.57... -> 9586981 = 0x924925
+    const float r = __uint_as_float(0x3B124925u);
     const float q0 = __fmul_rn(amax, r);
     const float e = __fmaf_rn(-q0, 448.0f, amax);
     return __fmaf_rn(e, r, q0);

@@ -247,10 +247,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
       const ScaleDivider d(sc);
       // this thread's first row and its outputs; rows i step by kQThreads / 16
       const int64_t r0 = rb * 128 + (t >> 4);
-      const int rows_here = static_cast<int>(a.rows - r0 < 0 ? 0 : a.rows - r0);
-#pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        if (i * (kQThreads / 16) >= rows_here) break;
+      auto row = [&](int i) {
         const int64_t r = r0 + i * (kQThreads / 16);
         if constexpr (kMode == QMode::kWeight) {
           reinterpret_cast<uint2*>(a.q + r * a.K + kb * 128)[chunk] = encode8_sign_merged(v[i], d);
@@ -263,6 +260,18 @@ __global__ void __launch_bounds__(kQThreads, 2)
           reinterpret_cast<uint32_t*>(a.q + r * (a.K / 2) + kb * 64)[chunk] = packed;
           a.meta[r * (a.K / 8) + kb * 16 + chunk] = static_cast<uint8_t>(meta);
           if constexpr (kOut) reinterpret_cast<uint4*>(a.pruned + r * a.K + kb * 128)[chunk] = pr;
+        }
+      };
+      if ((rb + 1) * 128 <= a.rows) {
+        // a whole row block (the same branch for the CTA): no row checks
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) row(i);
+      } else {
+        const int rows_here = static_cast<int>(a.rows - r0 < 0 ? 0 : a.rows - r0);
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          if (i * (kQThreads / 16) >= rows_here) break;
+          row(i);
         }
       }
     }

@@ -320,64 +320,85 @@ cudaError_t launch_stream(const void* x, int64_t rows, int64_t K, QArgs a, cudaS
   return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
-// Activation quantization (S1). A team of 16 threads quantizes 1x128
-// groups: each thread one 16-byte chunk (8 bf16) of a group, a 16-lane
-// shuffle max, the encode of e4m3_codec.cuh, one 8-byte store; the team's
-// first thread writes the scale. A team takes kGroups groups spread over the
-// grid (team, team + teams, ...) and issues all their loads before any
-// arithmetic: 4 for inputs that fill the GPU many times over (64 bytes per
-// thread in flight), 1 for decode-sized inputs (lowest latency). Groups are
+// Activation quantization (S1). A team of kTeam threads quantizes 1x128
+// groups: each thread 128 / kTeam adjacent bf16 of a group (one or two
+// 16-byte chunks), a kTeam-lane shuffle max, the encode of e4m3_codec.cuh,
+// one store of its codes; the team's first thread writes the scale. A team
+// takes kGroups groups spread over the grid (team, team + teams, ...) and
+// issues all their loads before any arithmetic. Inputs that fill the GPU many
+// times over use teams of 8 and 4 groups (128 bytes per thread in flight):
+// with one chunk per thread the per-group work (the shuffle max, the scale
+// and its divider) cost as many instructions as the codes and made the
+// kernel ALU-bound (8192 x 14336: 62.1 -> 51.6 us); mid-sized inputs use
+// teams of 8 with one group. Inputs of up to 8192 groups use teams of 16 and
+// one group (the shortest path per thread, the lowest latency). Groups are
 // contiguous in memory (row-major [M][K], K a multiple of 128) and the scale
 // of group g is sa[g] (row-major [M][K/128]). No shared memory and no
 // barrier: for decode-sized inputs the kernel costs one load round trip.
 constexpr int kActThreads = 256;
 
-template <int kGroups, bool kE8 = false>
+template <int kGroups, int kTeam, bool kE8 = false>
 __global__ void __launch_bounds__(kActThreads)
     act_quant_kernel(const __nv_bfloat16* __restrict__ x, int64_t groups,
                      uint8_t* __restrict__ q, void* __restrict__ scale) {
+  static_assert(kTeam == 8 || kTeam == 16, "one or two 16-byte chunks per thread");
+  constexpr int kChunks = 16 / kTeam;   // 16-byte chunks per thread
   // kE8: UE8M0 (power-of-two) scales, written as one code byte per group
-  const int64_t teams = static_cast<int64_t>(gridDim.x) * (kActThreads / 16);
-  const int64_t team = static_cast<int64_t>(blockIdx.x) * (kActThreads / 16) + (threadIdx.x >> 4);
-  const int chunk = threadIdx.x & 15;
+  const int64_t teams = static_cast<int64_t>(gridDim.x) * (kActThreads / kTeam);
+  const int64_t team =
+      static_cast<int64_t>(blockIdx.x) * (kActThreads / kTeam) + (threadIdx.x / kTeam);
+  const int part = threadIdx.x % kTeam;   // this thread's chunks: kChunks * part ...
   // While the previous kernel of the stream may still run, bring this
   // thread's input lines into L2 (one thread per 128-byte line): the
   // prefetch never changes what the loads below read, even if that kernel
   // writes x, and when it does not, the HBM latency overlaps the wait.
-  if ((chunk & 7) == 0) {
+  if ((part * kChunks) % 8 == 0) {
 #pragma unroll
     for (int j = 0; j < kGroups; ++j) {
       const int64_t g = team + j * teams;
-      if (g < groups) prefetch_l2(reinterpret_cast<const uint4*>(x + g * 128) + chunk);
+      if (g < groups) prefetch_l2(reinterpret_cast<const uint4*>(x + g * 128) + kChunks * part);
     }
   }
   grid_dependency_wait();
   grid_launch_dependents();
-  uint4 v[kGroups];
+  uint4 v[kGroups][kChunks];
 #pragma unroll
   for (int j = 0; j < kGroups; ++j) {
     const int64_t g = team + j * teams;
-    v[j] = g < groups ? __ldg(reinterpret_cast<const uint4*>(x + g * 128) + chunk)
-                      : make_uint4(0u, 0u, 0u, 0u);
+    const uint4* src = reinterpret_cast<const uint4*>(x + g * 128) + kChunks * part;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c)
+      v[j][c] = g < groups ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int j = 0; j < kGroups; ++j) {
     const int64_t g = team + j * teams;
-    float m = absmax_to_float(absmax8(v[j]));
+    uint32_t m2 = absmax8(v[j][0]);
 #pragma unroll
-    for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int c = 1; c < kChunks; ++c) m2 = bf16x2_absmax(m2, absmax8(v[j][c]));
+    float m = absmax_to_float(m2);
+#pragma unroll
+    for (int off = kTeam / 2; off >= 1; off >>= 1)
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    uint2 c8[kChunks];
     if constexpr (kE8) {
       const uint32_t code = ue8m0_code_of_amax(m);
-      if (g < groups) {
-        reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8_pow2(v[j], ue8m0_inv_scale(code));
-        if (chunk == 0) static_cast<uint8_t*>(scale)[g] = static_cast<uint8_t>(code);
-      }
+      const float inv = ue8m0_inv_scale(code);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) c8[c] = encode8_pow2(v[j][c], inv);
+      if (g < groups && part == 0) static_cast<uint8_t*>(scale)[g] = static_cast<uint8_t>(code);
     } else {
       const float sc = scale_of_amax(m);
-      if (g < groups) {
-        reinterpret_cast<uint2*>(q + g * 128)[chunk] = encode8(v[j], ScaleDivider(sc));
-        if (chunk == 0) static_cast<float*>(scale)[g] = sc;
-      }
+      const ScaleDivider d(sc);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) c8[c] = encode8(v[j][c], d);
+      if (g < groups && part == 0) static_cast<float*>(scale)[g] = sc;
+    }
+    if (g < groups) {
+      if constexpr (kChunks == 2)
+        reinterpret_cast<uint4*>(q + g * 128)[part] = make_uint4(c8[0].x, c8[0].y, c8[1].x, c8[1].y);
+      else
+        reinterpret_cast<uint2*>(q + g * 128)[part] = c8[0];
     }
   }
 }
@@ -392,11 +413,14 @@ cudaError_t launch_act(const void* x, int64_t M, int64_t K, void* qa, void* sa,
   DeviceInfo dev;
   if (current_device_info(&dev) != FP8BS_OK) return cudaErrorInvalidDevice;
   const int64_t groups = M * (K / 128);
-  const int64_t teams_per_block = kActThreads / 16;
-  // one group per team unless one team per group would fill every SM
-  // (2048 threads) eight times over
-  const int per = groups >= 8LL * dev.sm_count * (2048 / 16) ? 4 : 1;
-  const int64_t blocks = (groups + teams_per_block * per - 1) / (teams_per_block * per);
+  // teams of 16 with one group each for the smallest inputs (up to 8192
+  // groups: the shortest path per thread); teams of 8, with four groups each
+  // once teams of 8 would fill every SM (2048 threads) eight times over, else
+  // with one
+  const int form = groups <= 8192 ? 0 : groups >= 8LL * dev.sm_count * (2048 / 8) ? 2 : 1;
+  const int64_t per_block = form == 0 ? kActThreads / 16 : form == 1 ? kActThreads / 8
+                                                                     : (kActThreads / 8) * 4;
+  const int64_t blocks = (groups + per_block - 1) / per_block;
   if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
@@ -409,8 +433,9 @@ cudaError_t launch_act(const void* x, int64_t M, int64_t K, void* qa, void* sa,
   cfg.numAttrs = 1;
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* qp = static_cast<uint8_t*>(qa);
-  return per == 4 ? cudaLaunchKernelEx(&cfg, act_quant_kernel<4, kE8>, xp, groups, qp, sa)
-                  : cudaLaunchKernelEx(&cfg, act_quant_kernel<1, kE8>, xp, groups, qp, sa);
+  if (form == 2) return cudaLaunchKernelEx(&cfg, act_quant_kernel<4, 8, kE8>, xp, groups, qp, sa);
+  if (form == 1) return cudaLaunchKernelEx(&cfg, act_quant_kernel<1, 8, kE8>, xp, groups, qp, sa);
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<1, 16, kE8>, xp, groups, qp, sa);
 }
 
 }  // namespace

@@ -12,9 +12,10 @@
 // The tile kernel (S2, S4) streams HBM. CTAs are persistent (two per SM); thread
 // 0 keeps a 3-deep ring of 32 KB tiles in flight with TMA
 // (cp.async.bulk.tensor, no swizzle, out-of-range rows read as zero), and all
-// 512 threads work from shared memory. Thread t owns the 16-byte chunk t % 16
-// of rows t/16 + 32 i (i = 0..3): 16 threads cover one 256-byte row, so every
-// global store of a warp is contiguous. The element quotient x / s is the IEEE
+// T threads (512 for weight blocks, 256 for 2:4) work from shared memory.
+// Thread t owns the 16-byte chunk t % 16 of rows t/16 + (T/16) i (i < 2048/T):
+// 16 threads cover one 256-byte row, so every global store of a warp is
+// contiguous. The element quotient x / s is the IEEE
 // fp32 quotient (ScaleDivider) and the conversion is the hardware
 // cvt.rn.satfinite.e4m3x2.f32.
 #include <mutex>
@@ -32,8 +33,16 @@ enum class QMode { kWeight, kPrune, kPruneOut, kWeightE8 };
 
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kQStages = 3;
-constexpr int kQThreads = 512;
-constexpr int kRowsPerThread = 128 * 16 / kQThreads;   // 16 threads per 256-byte row
+// Threads per CTA: 256 for the 2:4 modes (8 rows per thread, so the per-tile
+// work -- the block max, the scale and its divider -- is spread over twice as
+// many values: 28672 x 4096 59.8 -> 55.7 us), 512 for the weight blocks (4
+// rows per thread; 56.2 against 58.4 us with 256).
+template <QMode kMode>
+struct QCfg {
+  static constexpr int kThreads =
+      (kMode == QMode::kPrune || kMode == QMode::kPruneOut) ? 256 : 512;
+  static constexpr int kRowsPerThread = 128 * 16 / kThreads;   // 16 threads per 256-byte row
+};
 constexpr int kQSmemBytes = kQStages * kTileBytes + 1024 + 64;
 
 struct QArgs {
@@ -123,8 +132,10 @@ __device__ __forceinline__ uint32_t prune8(const uint4 v, const ScaleDivider& d,
 }
 
 template <QMode kMode>
-__global__ void __launch_bounds__(kQThreads, 2)
+__global__ void __launch_bounds__(QCfg<kMode>::kThreads, 2)
     stream_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const QArgs a) {
+  constexpr int kQThreads = QCfg<kMode>::kThreads;
+  constexpr int kRowsPerThread = QCfg<kMode>::kRowsPerThread;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -309,7 +320,7 @@ cudaError_t launch_stream(const void* x, int64_t rows, int64_t K, QArgs a, cudaS
   const int64_t ctas = a.num_tiles < 2LL * dev.sm_count ? a.num_tiles : 2LL * dev.sm_count;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.blockDim = dim3(QCfg<kMode>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kQSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute pdl;

@@ -43,17 +43,27 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
   alignas(64) CUtensorMap ta, tb;
 
   const uint64_t KB = static_cast<uint64_t>(K / 128);
-  if (decode_order(M, N, dev.sm_count) && qy != nullptr) {
-    // Decode-sized M with the next layer's quantization: Y, then the
-    // activation quantizer on it (the decode-order tile holds a group of N
-    // across four warps, or across a cluster with a K split).
+  // The next layer's quantization is fused into the epilogue for up to 16
+  // tokens in decode order when the tiles are not split over K (a group of N
+  // is a tile's 128 weight rows, staged per token for the Y stores), and above
+  // 256 tokens in prefill order (a thread holds a group). In between, and with
+  // a K split (a group spans the cluster), Y is written and then quantized by
+  // the activation quantizer: timed on gate+up (28672 x 4096), the epilogue's
+  // quantization sits on the last tile's critical path and cost more than the
+  // second launch from 32 tokens on (64 tokens: 30.8 against 29.1 us; 128, in
+  // prefill order: 30.2 against 29.5 us), and saved 0.6 us at 1 and 8.
+  const bool decode = decode_order(M, N, dev.sm_count);
+  const bool fuse_decode = decode && qy != nullptr && M <= 16 &&
+                           choose_splits(static_cast<int>((N + 127) / 128), dev.sm_count,
+                                         a.KB, 2) == 1;
+  if (qy != nullptr && M <= 256 && !fuse_decode) {
     if (int st = launch_block_gemm(qa, sa, qw, sw, y, M, N, K, wait_limit, err, stream, nullptr,
                                    nullptr))
       return st;
     return launch_quant_act_group128(y, M, N, qy, sy, stream) == cudaSuccess ? FP8BS_OK
                                                                               : FP8BS_ERR_CUDA;
   }
-  if (decode_order(M, N, dev.sm_count)) {
+  if (decode) {
     // Decode: weights on the MMA M side, tokens on the MMA N side; stages of
     // two K-blocks.
     constexpr int kKS = 2;
@@ -66,6 +76,8 @@ int launch_block_gemm(const void* qa, const float* sa, const void* qw, const flo
     const int grid_y = S > 1 ? tiles : (tiles < dev.sm_count ? tiles : dev.sm_count);
     if (int st = encode_tmap_kblocks(&ta, qw, 128, N, KB, K, 128, kKS, kSwizzle128B)) return st;
     if (int st = encode_tmap_kblocks(&tb, qa, 128, M, KB, K, BN, kKS, kSwizzle128B)) return st;
+    if (fuse_decode)   // BN == 16 and S == 1 here
+      return launch_cfg<16, true, false, 5, 1, kKS, true>(ta, tb, ta, a, grid_y, 1, stream);
     switch (BN) {
       case 16: return launch_cfg<16, true, false, 5, 1, kKS>(ta, tb, ta, a, grid_y, S, stream);
       case 32: return launch_cfg<32, true, false, 5, 1, kKS>(ta, tb, ta, a, grid_y, S, stream);

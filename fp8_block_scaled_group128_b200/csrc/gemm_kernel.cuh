@@ -204,11 +204,14 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
                       const __grid_constant__ CUtensorMap tmap_e,
                       const __grid_constant__ CUtensorMap tmap_y, const GemmArgs args) {
   // tmap_e: the 2:4 metadata (sparse only); tmap_y: the output Y for the TMA
-  // stores of the epilogue. kQOut (prefill order only): the epilogue also
-  // quantizes Y for the next layer (args.qy, args.sy) and Y itself is written
-  // only if args.y is set.
+  // stores of the epilogue. kQOut: the epilogue also quantizes Y for the next
+  // layer (args.qy, args.sy); in prefill order each thread holds one 1x128
+  // group and Y itself is written only if args.y is set; in decode order
+  // (unsplit tiles only) each token's group is the tile's 128 weight rows,
+  // quantized from the staging buffer of the Y stores.
   using C = Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>;
-  static_assert(!kQOut || (!kSwap && C::kCols == 128), "fused quantization: one group per thread");
+  static_assert(!kQOut || (!kSparse && (kSwap || C::kCols == 128)),
+                "fused quantization: one group per thread or per staged token");
   // kSwiGLU (prefill order): the 256 weight rows of a tile are gate rows
   // [128 ct, 128 ct + 128) and up rows [I + 128 ct, ...) (two TMA boxes of 128
   // rows); warpgroup 0 promotes the gate columns, warpgroup 1 the up columns of
@@ -783,9 +786,34 @@ __global__ void __launch_bounds__(Cfg<BN, kSwap, kSparse, kStages, kEpiWG, kKS>:
           }
           fence_proxy_async_smem();
           named_bar_sync(2 + wg, 128);
-          if (leader && ok) {
+          if (leader && ok && (!kQOut || args.y != nullptr)) {
             tma_store_2d(&tmap_y, stage_y, rt * 128, ct * BN + col0 + c);
             bulk_commit_group();
+          }
+          if constexpr (kQOut) {
+            // Each staged token holds one whole 1x128 group of Y (the tile's
+            // 128 weight rows, 256 contiguous bytes): a team of 16 threads per
+            // token quantizes it with the activation quantizer's arithmetic
+            // (8 bf16 per thread, a 16-lane max) and writes 128 code bytes and
+            // the scale. The staging buffer is rewritten only after the next
+            // chunk's barrier, which every thread reaches after these reads.
+            const int part = (warp & 3) * 32 + lane;
+            const int team = part >> 4, sub = part & 15;
+#pragma unroll
+            for (int j = team; j < C::kChunk; j += 8) {
+              const uint4 v = *reinterpret_cast<const uint4*>(stage_y + j * 256 + sub * 16);
+              float am = absmax_to_float(absmax8(v));
+#pragma unroll
+              for (int off = 8; off >= 1; off >>= 1)
+                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+              const float sc = scale_of_amax(am);
+              const int64_t m = static_cast<int64_t>(ct) * BN + col0 + c + j;   // token
+              if (ok && m < args.M) {
+                *reinterpret_cast<uint2*>(args.qy + m * args.N + rt * 128 + sub * 8) =
+                    encode8(v, ScaleDivider(sc));
+                if (sub == 0) args.sy[m * (args.N / 128) + rt] = sc;
+              }
+            }
           }
         }
       }

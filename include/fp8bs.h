@@ -133,10 +133,11 @@ int fp8_block_gemm(const void* qa, const float* sa, const void* qw, const float*
  * y, and qy / sy = fp8_quant_act_group128(y) of that bf16 y, i.e. y's rows
  * cut into 1x128 groups along N ("FP8 à granularité fine": the output of one
  * linear is the activation of the next, quantized per token per 128
- * channels). When the GEMM runs in prefill order (M > 256, or M > 64 with N
- * wide enough to fill most of the GPU with 128 x 256 tiles) its epilogue
- * quantizes its own tile (each promotion thread holds one group); otherwise
- * y is written and then quantized by the activation quantizer.
+ * channels). For M > 256 the GEMM's epilogue quantizes its own tile (each
+ * promotion thread holds one group); for M <= 16 with unsplit decode tiles
+ * (N of at least 75 row blocks on 148 SMs) the decode-order epilogue
+ * quantizes each token's staged group; otherwise y is written and then
+ * quantized by the activation quantizer.
  *
  *   y_bf16  [M][N] bf16, output; may be NULL when M > 256 (then only the codes
  *           are written), required when M <= 256.

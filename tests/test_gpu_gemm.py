@@ -176,12 +176,12 @@ def test_operand_order_boundary_wide_n(M):
 
 @pytest.mark.parametrize("M,N", [(65, 28672), (200, 14208), (128, 28288), (128, 28160)])
 def test_fused_quantization_in_prefill_order_at_decode_sizes(M, N):
-    """fp8_block_gemm_quant for 65..256 tokens on wide weights. On 148 SMs:
-    N = 28288 at M = 128 is the narrowest width that takes the one-kernel
-    prefill-order form (111 tiles of 128 x 256) and 28160 the widest that
-    stays in decode order (GEMM, then the quantizer); 28288 and 14208 (M = 200,
-    two row tiles) leave the last 256-column tile half empty. y equal to
-    fp8_block_gemm's, codes and scales equal to the oracle's quantization of
+    """fp8_block_gemm_quant for 65..256 tokens on wide weights: the GEMM in
+    either operand order, then the quantizer. On 148 SMs N = 28288 at M = 128
+    is the narrowest width whose GEMM runs in prefill order (111 tiles of
+    128 x 256) and 28160 the widest that stays in decode order; 28288 and 14208
+    (M = 200, two row tiles) leave the last 256-column tile half empty. y equal
+    to fp8_block_gemm's, codes and scales equal to the oracle's quantization of
     that y."""
     K = 384
     qa, sa, qw, sw = _quantized("llama", M, N, K, 5)
@@ -273,13 +273,20 @@ def test_bounded_wait_reports_timeout_and_recovers(M):
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 4096, 4096), (128, 6144, 4096), (300, 640, 512),
-                                   (2048, 6144, 4096), (4096, 2048, 1024), (8192, 4096, 14336)])
+                                   (2048, 6144, 4096), (4096, 2048, 1024), (8192, 4096, 14336),
+                                   (1, 28672, 4096), (8, 9600, 512), (16, 14336, 384),
+                                   (37, 14336, 384), (64, 28672, 256), (100, 12288, 512),
+                                   (128, 28160, 384)])
 def test_gemm_with_fused_next_layer_quantization(M, N, K):
     """fp8_block_gemm_quant gives fp8_block_gemm's y, byte for byte, and the
     next layer's 1x128 codes and scales of that bf16 y exactly as the oracle's
     activation quantizer computes them; with M > 256 (the fused epilogue) also
     when y itself is not written. N = 640 leaves the second warpgroup of the
-    last column tile without a group."""
+    last column tile without a group. Up to 16 tokens with at least 75 row
+    tiles (N >= 9600) the decode-order tiles run unsplit and quantize in the
+    epilogue from the staged Y (M = 1, 8, 16); 17..256 tokens, and the split
+    shapes (4096 and 6144 rows), write Y and run the quantizer (M = 37, 64,
+    100, 128)."""
     qa, sa, qw, sw = _quantized("llama", M, N, K, 3)
     args = [to_dev(a) for a in (qa, sa, qw, sw)]
     y_plain = fb.fp8_block_gemm(*args)

@@ -232,9 +232,10 @@ int fp8_grouped_gemm_ue8m0(const void* qa, const uint8_t* sa_ue8m0, const void* 
  *       aligned (required for M <= 256 only, else may be NULL): there the
  *       call may run the decode-order GEMM of the 2I weight rows into this
  *       scratch (g and u rounded to bf16) and a second kernel that forms h and
- *       its codes; otherwise (M > 256, or a 2I wide enough for the prefill
- *       order as in fp8_block_gemm_quant) one kernel does all of it from the
- *       fp32 accumulators. Both forms meet the same tolerance on h.
+ *       its codes; otherwise (M > 256, or M > 64 with 2I wide enough that
+ *       tiles of 128 tokens x 256 weight rows fill at least three quarters of
+ *       the GPU) one kernel does all of it from the fp32 accumulators. Both
+ *       forms meet the same tolerance on h.
  *   I must be a positive multiple of 128. Same errors as fp8_block_gemm;
  *   FP8BS_ERR_WORKSPACE for a missing or short workspace.
  */

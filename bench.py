@@ -401,15 +401,21 @@ def run_prefill(dev, stream, world, reps=12):
     # plain gate+up GEMM of the same shape is the dense row (or timed here)
     shapes += [(kind, M, 28672, 4096) for M in (8, 128) for kind in ("swiglu", "dense")]
     shapes += [("swiglu", M, 28672, 4096) for M in synth.PREFILL_M]
-    rows, tot = [], {"dense": [0.0, 0.0], "ue8m0": [0.0, 0.0]}
+    shapes = [sh + ("llama",) for sh in shapes]
+    # the DeepSeek-V3 linears (their own weight and activation statistics) at
+    # M = 4096, both scale formats
+    shapes += [(kind, 4096, N, K, "deepseek") for N, K in synth.DEEPSEEK_V3_LINEARS
+               for kind in ("dense", "ue8m0")]
+    rows = []
+    tot = {g: [0.0, 0.0] for g in ("dense", "ue8m0", "ds_dense", "ds_ue8m0")}
     wcache = {}
-    for kind, M, N, K in shapes:
+    for kind, M, N, K, wl in shapes:
         with torch.cuda.stream(stream):
-            key = (N, K)
+            key = (wl, N, K)
             if key not in wcache:
                 wcache.clear()
                 torch.cuda.empty_cache()
-                wcache[key] = synth.weights("llama", N, K, seed=7).to(dev)
+                wcache[key] = synth.weights(wl, N, K, seed=7).to(dev)
             w = wcache[key]
             if kind == "sparse":
                 wq = list(fb.prune24_compress(w)[:3])
@@ -417,7 +423,7 @@ def run_prefill(dev, stream, world, reps=12):
                 wq = list(fb.fp8_quant_weight_block128_ue8m0(w))
             else:
                 wq = list(fb.fp8_quant_weight_block128(w))
-            x = synth.activations("llama", M, K, seed=7).to(dev)
+            x = synth.activations(wl, M, K, seed=7).to(dev)
             qa, sa = (fb.fp8_quant_act_group128_ue8m0(x) if kind == "ue8m0"
                       else fb.fp8_quant_act_group128(x))
             del x
@@ -454,11 +460,13 @@ def run_prefill(dev, stream, world, reps=12):
         # algorithmic FLOPs: 2MNK dense; MNK (the kept half) for 2:4
         flop = (1.0 if kind == "sparse" else 2.0) * M * N * K
         tf = flop / (ms * 1e-3) / 1e12
-        rows.append({"gemm": kind, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1),
-                     "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4), "input_copies": n_cp})
-        if kind in tot and M in synth.PREFILL_M:
-            tot[kind][0] += flop
-            tot[kind][1] += ms
+        rows.append({"gemm": kind, "workload": wl, "M": M, "N": N, "K": K,
+                     "us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
+                     "input_copies": n_cp})
+        group = kind if wl == "llama" else "ds_" + kind
+        if group in tot and (wl != "llama" or M in synth.PREFILL_M):
+            tot[group][0] += flop
+            tot[group][1] += ms
         del fns, ins, qa, sa, wq, y, qy, sy, qh_sw, sh_sw
     wcache.clear()
     torch.cuda.empty_cache()
@@ -467,15 +475,19 @@ def run_prefill(dev, stream, world, reps=12):
     return {"bound": "tensor", "unit": "TFLOP/s", "peak": round(peak, 1), "peak_source": peak_src,
             "dense_achieved": round(agg["dense"], 1), "dense_frac": round(agg["dense"] / peak, 4),
             "ue8m0_achieved": round(agg["ue8m0"], 1), "ue8m0_frac": round(agg["ue8m0"] / peak, 4),
+            "deepseek_dense_achieved": round(agg["ds_dense"], 1),
+            "deepseek_dense_frac": round(agg["ds_dense"] / peak, 4),
+            "deepseek_ue8m0_achieved": round(agg["ds_ue8m0"], 1),
+            "deepseek_ue8m0_frac": round(agg["ds_ue8m0"] / peak, 4),
             "note": "dense: fp32 scales (per-K-block promotion), 2MNK FLOPs; ue8m0: power-of-two "
-                    "scales applied by the block-scaled MMA; 2:4: MNK FLOPs (nonzero work) against "
-                    "the dense peak; fused / separate: the down projection with the next layer's "
-                    "1x128 quantization in the epilogue / after it (M = 8192; at M <= 256 the "
-                    "fused entry point runs the GEMM and then the quantizer, two launches; not "
-                    "in dense_achieved); swiglu: gate+up GEMM with SwiGLU and the down "
-                    "projection's quantization (codes only; one kernel above 256 tokens, GEMM + "
-                    "SwiGLU kernel at or below), against the plain gate+up GEMM; inputs "
-                    "rotated over copies so that none is in L2 at its launch",
+                    "scales applied by the block-scaled MMA; dense/ue8m0_achieved average the "
+                    "llama prefill shapes, deepseek_* the DeepSeek-V3 linears at M = 4096; 2:4: "
+                    "MNK FLOPs (nonzero work) against the dense peak; fused / separate: the down "
+                    "projection with the next layer's 1x128 quantization in the epilogue / after "
+                    "it (M = 8192; not in dense_achieved); swiglu: gate+up GEMM with SwiGLU and "
+                    "the down projection's quantization (codes only; one kernel where the gate+up "
+                    "GEMM runs in prefill order, here M > 64), against the plain gate+up GEMM; "
+                    "inputs rotated over copies so that none is in L2 at its launch",
             "shapes": rows}
 
 

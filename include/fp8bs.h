@@ -250,10 +250,11 @@ size_t fp8bs_swiglu_workspace_bytes(int64_t M, int64_t I);
 /*
  * fp8_gemm_swiglu_quant without a workspace and without any device allocation
  * (no cudaMalloc / cudaFree, no allocating library call). The paper (the
- * pages this library follows) has no counterpart: it exists for callers that cannot hand over or obtain device
- * memory per call, such as a C host that owns every buffer and passes only
- * operands in and out (a plugin or custom-op interface with no workspace
- * slot), or a decode loop that must not enter an allocator because
+ * pages this library follows) has no counterpart: it exists for callers that
+ * cannot hand over or obtain device memory per call, such as a C host that
+ * owns every buffer and passes only operands in and out (a plugin or
+ * custom-op interface with no workspace slot), or a decode loop that must not
+ * enter an allocator because
  * cudaMalloc / cudaFree may synchronise the device and fail once a memory
  * pool has reserved the free memory.
  *
